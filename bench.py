@@ -1,0 +1,600 @@
+#!/usr/bin/env python
+"""Throughput of the next-token cross-entropy hot path on B200.
+
+One JSON line (rank 0).  Default workload: standalone CE forward+backward on
+GPT-2-shaped bf16 logits [8192, 50257] (2% ignored, mean, z-loss 1e-4); the
+same line carries the chunked linear-CE on the GPT-2 small tied head
+([8192, 768] x [50257, 768], chunk 2048, fp32 accumulation) under "linear_ce".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
+
+Timing: CUDA events on the launching stream around exactly K steps, bracketed
+by a barrier and a device synchronise, max over ranks.  Inputs are larger than
+L2 (126 MB) for the timed workloads, so no flush runs between steps.  Kernel
+durations for the roofline come from libgh's own event pairs around the
+dominant kernel, recorded during the same timed region.  With N > 1 each rank
+processes its own batch (seed = rank); nothing is exchanged (weak scaling).
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CE tokens/s and HBM GB/s; linear-CE tokens/s and TFLOP/s vs bf16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+CE_WORKLOADS = {"ce_gpt2": "ce_gpt2", "ce_large_vocab": "ce_large_vocab", "ce_small": "ce_small"}
+LINEAR_WORKLOADS = {"linear_ce_gpt2": "linear_ce_gpt2", "linear_ce_llama3_8b": "linear_ce_llama3_8b"}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest(files):
+    h = hashlib.sha1()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(summary_file, digest, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+    p = os.path.join(ROOT, "profiles", summary_file)
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", txt)
+    m_wl = re.search(r"workload:\s*(\S+)", txt)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not (m_sha and m_tr and m_wl) or m_sha.group(1) != digest or m_wl.group(1) != workload:
+        return None
+    return float(m_tr.group(1))
+
+
+# --------------------------------------------------------------------------
+# clocks
+# --------------------------------------------------------------------------
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+           0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+           0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML in a thread."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nvml, self._h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.period = period_s
+        self._t = None
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+                try:
+                    r = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    r = n.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((sm, int(r)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = statistics.median(s for s, _ in self.samples)
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = sorted(name for b, name in REASONS.items() if bits & b and name != "gpu_idle")
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend="nccl"):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch
+            import torch.distributed as dist
+            dist.barrier(device_ids=[torch.cuda.current_device()]) if dist.get_backend() == "nccl" else dist.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# workloads
+# --------------------------------------------------------------------------
+
+ROWS = 0  # --rows: truncate the batch (profiling cases only)
+
+
+def make_ce(name, seed):
+    import gh_synth
+    p = getattr(gh_synth, CE_WORKLOADS[name])(seed=seed) if name != "ce_small" else gh_synth.ce_small(1e-4, seed)
+    if ROWS:
+        p.logits = p.logits[:ROWS].copy()
+        p.targets = p.targets[:ROWS].copy()
+        p.name += f"_rows{ROWS}"
+    return p
+
+
+def make_linear(name, seed):
+    import gh_synth
+    p = getattr(gh_synth, LINEAR_WORKLOADS[name])(seed=seed)
+    if ROWS:
+        p.inputs = p.inputs[:ROWS].copy()
+        p.targets = p.targets[:ROWS].copy()
+        p.name += f"_rows{ROWS}"
+    return p
+
+
+def pinned(a):
+    import numpy as np
+    import torch
+    if a.dtype == np.uint16:
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(a)
+    return t.pin_memory()
+
+
+class CeCase:
+    kind = "ce"
+
+    def __init__(self, name, seed, dev):
+        import numpy as np
+        import torch
+        self.p = make_ce(name, seed)
+        self.h_x = pinned(self.p.logits)
+        self.h_t = pinned(self.p.targets)
+        self.x = self.h_x.to(dev, non_blocking=False)
+        self.t = self.h_t.to(dev)
+        self.grad = torch.empty_like(self.x)
+        self.loss = torch.empty((), dtype=torch.float32, device=dev)
+        self.h_loss = torch.empty((), dtype=torch.float32).pin_memory()
+        self.tokens = self.p.B
+        es = 4 if self.p.dtype == "f32" else 2
+        n_ign = int((self.p.targets == self.p.ignore_index).sum())
+        # algorithmic bytes: read every valid row once, write every gradient row once, read targets
+        self.bytes_per_step = ((self.p.B - n_ign) * self.p.V + self.p.B * self.p.V) * es + 8 * self.p.B
+        self.h2d = self.h_x.numel() * self.h_x.element_size() + self.h_t.numel() * 8
+        self.d2h = 4
+        self.dtype = "bf16" if self.p.dtype == "bf16" else "f32"
+
+    def step(self):
+        import lm_head_cross_gh_b200 as gh
+        p = self.p
+        gh.gh_ce_fwd_bwd(self.x, self.t, p.ignore_index, p.reduction, p.z_loss, grad=self.grad, loss=self.loss)
+
+    def e2e_step(self):
+        import lm_head_cross_gh_b200 as gh
+        p = self.p
+        self.x.copy_(self.h_x, non_blocking=True)
+        self.t.copy_(self.h_t, non_blocking=True)
+        gh.gh_ce_fwd_bwd(self.x, self.t, p.ignore_index, p.reduction, p.z_loss, grad=self.grad, loss=self.loss)
+        self.h_loss.copy_(self.loss, non_blocking=True)
+
+    def config(self):
+        p = self.p
+        return {"workload": p.name, "B": p.B, "V": p.V, "dtype": p.dtype, "reduction": p.reduction,
+                "z_loss": p.z_loss, "ignore_index": p.ignore_index,
+                "ignored_rows": int((p.targets == p.ignore_index).sum()),
+                "l2": f"inputs larger than L2 ({p.B * p.V * (4 if p.dtype == 'f32' else 2) / 1e6:.0f} MB); no flush"}
+
+    def cpu_sample(self, budget_rows):
+        import numpy as np
+        p = self.p
+        rows = np.arange(min(p.B, budget_rows))
+        return rows
+
+    def run_oracle(self, rows):
+        import numpy as np
+        import oracle
+        p = self.p
+        _, scale = oracle.n_valid_and_scale(p.targets, p.ignore_index, p.reduction, p.V)
+        oracle.ce_rows(p.values_f32(rows).astype(np.float64), p.targets[rows], p.ignore_index, p.z_loss, scale)
+        return len(rows)
+
+
+class LinearCase:
+    kind = "linear"
+
+    def __init__(self, name, seed, dev):
+        import torch
+        self.p = make_linear(name, seed)
+        self.h_X = pinned(self.p.inputs)
+        self.h_W = pinned(self.p.weight)
+        self.h_t = pinned(self.p.targets)
+        self.X = self.h_X.to(dev)
+        self.W = self.h_W.to(dev)
+        self.t = self.h_t.to(dev)
+        self.dX = torch.empty_like(self.X)
+        self.dW = torch.empty_like(self.W)
+        self.loss = torch.empty((), dtype=torch.float32, device=dev)
+        self.h_loss = torch.empty((), dtype=torch.float32).pin_memory()
+        p = self.p
+        self.tokens = p.N
+        self.flops_per_step = 6.0 * p.N * p.V * p.D
+        self.h2d = (self.h_X.numel() + self.h_W.numel()) * 2 + self.h_t.numel() * 8
+        self.d2h = 4
+        self.dtype = "bf16"
+
+    def step(self):
+        import lm_head_cross_gh_b200 as gh
+        p = self.p
+        gh.gh_linear_ce(self.X, self.W, self.t, p.ignore_index, p.reduction, p.z_loss, p.chunk, p.accum,
+                        grad_inputs=self.dX, grad_weight=self.dW, loss=self.loss)
+
+    def e2e_step(self):
+        import lm_head_cross_gh_b200 as gh
+        p = self.p
+        self.X.copy_(self.h_X, non_blocking=True)
+        self.W.copy_(self.h_W, non_blocking=True)
+        self.t.copy_(self.h_t, non_blocking=True)
+        gh.gh_linear_ce(self.X, self.W, self.t, p.ignore_index, p.reduction, p.z_loss, p.chunk, p.accum,
+                        grad_inputs=self.dX, grad_weight=self.dW, loss=self.loss)
+        self.h_loss.copy_(self.loss, non_blocking=True)
+
+    def config(self):
+        p = self.p
+        return {"workload": p.name, "N": p.N, "D": p.D, "V": p.V, "chunk": p.chunk, "accum": p.accum,
+                "reduction": p.reduction, "z_loss": p.z_loss,
+                "ignored_rows": int((p.targets == p.ignore_index).sum()),
+                "l2": "weight and chunk logits larger than L2; no flush"}
+
+    def cpu_sample(self, budget_rows):
+        import numpy as np
+        return np.arange(min(self.p.N, budget_rows))
+
+    def run_oracle(self, rows):
+        """Oracle on a row sample: the chunk's logits, CE and both gradient GEMMs (float64)."""
+        import numpy as np
+        import gh_synth
+        import oracle
+        p = self.p
+        X = gh_synth.bf16_to_f32(p.inputs[rows]).astype(np.float64)
+        W = self._W64 if hasattr(self, "_W64") else gh_synth.bf16_to_f32(p.weight).astype(np.float64)
+        self._W64 = W
+        oracle.linear_cross_entropy(X, W, p.targets[rows], p.ignore_index, p.reduction, p.z_loss,
+                                    chunk=len(rows), accum=p.accum)
+        return len(rows)
+
+
+KERNEL_OF = {"ce": "ce_row", "linear": "logits_gemm"}
+
+
+def time_steps(case, dist, steps, warmup, clocks=None):
+    import torch
+    import lm_head_cross_gh_b200 as gh
+    for _ in range(warmup):
+        case.step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    kinds = ["ce_row"] if case.kind == "ce" else ["logits_gemm", "chunk_ce", "dx_gemm", "dw_gemm"]
+    gh.gh_profile_enable(True)
+    n0 = gh.gh_launch_count()
+    if clocks:
+        clocks.start()
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        case.step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    dist.barrier()
+    launches = gh.gh_launch_count() - n0
+    gh.gh_profile_enable(False)
+    # keep the clock record meaningful for short timed regions: the same work
+    # continues (untimed) until ~0.5 s of samples exist
+    if clocks:
+        pad_t = time.perf_counter()
+        while time.perf_counter() - pad_t < max(0.0, 0.5 - wall):
+            case.step()
+            torch.cuda.synchronize()
+        clocks.stop()
+    ms = e0.elapsed_time(e1)
+    kern = {}
+    for k in kinds:
+        tot, n = gh.gh_profile_read(k)
+        kern[k] = (tot, n)
+    return ms, launches, kern
+
+
+def time_e2e(case, dist, steps):
+    import torch
+    for _ in range(2):
+        case.e2e_step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        case.e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    return e0.elapsed_time(e1)
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        blas = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        return max(blas) if blas else 1
+    except Exception:
+        return 1
+
+
+def run_oracle_timing(case, budget_rows, reps=1):
+    rows = case.cpu_sample(budget_rows)
+    t0 = time.perf_counter()
+    n = 0
+    for _ in range(reps):
+        n += case.run_oracle(rows)
+    dt = time.perf_counter() - t0
+    return n / dt, len(rows), dt
+
+
+ORACLE_ROWS = {"ce_gpt2": 1024, "ce_large_vocab": 256, "ce_small": 64, "linear_ce_gpt2": 512,
+               "linear_ce_llama3_8b": 32}
+
+
+def linear_summary(case, ms, kern, steps, pk, peak_kind):
+    tot_ms = ms / steps
+    tflops = case.flops_per_step / (tot_ms * 1e-3) / 1e12
+    gemm_ms = sum(kern[k][0] for k in ("logits_gemm", "dx_gemm", "dw_gemm")) / steps
+    gemm_tflops = case.flops_per_step / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    return tot_ms, tflops, gemm_ms, gemm_tflops, peak
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="ce_gpt2", choices=list(CE_WORKLOADS) + list(LINEAR_WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-linear", action="store_true", help="omit the linear-CE object on the CE line")
+    ap.add_argument("--rows", type=int, default=0, help="use only the first ROWS rows/tokens (profiling cases)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    global ROWS
+    ROWS = max(0, args.rows)
+
+    dist = Dist()
+    if args.impl == "reference":
+        return reference_arm(args, dist)
+
+    import torch
+    import lm_head_cross_gh_b200 as gh
+    from lm_head_cross_gh_b200 import _build
+    if not os.path.exists(gh.LIB_PATH):
+        _build.build()
+    torch.cuda.set_device(dist.local)
+    dist.init("nccl")
+    dev = torch.device("cuda", dist.local)
+    pk, pk_kind = peaks()
+
+    is_ce = args.workload in CE_WORKLOADS
+    case = CeCase(args.workload, dist.rank, dev) if is_ce else LinearCase(args.workload, dist.rank, dev)
+    clocks = ClockSampler(dist.local)
+    ms, launches, kern = time_steps(case, dist, args.steps, args.warmup, clocks)
+    ms_max = dist.max(ms)
+    tokens_all = dist.sum(case.tokens * args.steps)
+    value = tokens_all / (ms_max * 1e-3)
+
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": case.dtype,
+           "data": "synthetic (seeded; seed = rank)", "config": case.config()}
+    out["config"]["parallelism"] = f"replicas x{dist.world} (independent batches, no collective)"
+
+    if is_ce:
+        k_ms, k_n = kern["ce_row"]
+        k_avg = k_ms / max(k_n, 1)
+        achieved = case.bytes_per_step / (k_avg * 1e-3) / 1e9
+        digest = source_digest(["lm_head_cross_gh_b200/csrc/ce.cu", "lm_head_cross_gh_b200/csrc/common.cuh"])
+        traffic = profiled_traffic("ce_row_kernel.md", digest, case.p.name)
+        out["roofline"] = {"bound": "hbm", "kernel": "ce_row_kernel", "achieved": achieved,
+                           "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                           "traffic": traffic, "algorithmic_bytes": case.bytes_per_step,
+                           "kernel_ms": k_avg, "peak_source": f"{pk_kind} (copy)", "source_sha": digest}
+        out["hbm_gbs_step"] = case.bytes_per_step * args.steps / (ms * 1e-3) / 1e9
+    else:
+        tot_ms, tflops, gemm_ms, gemm_tflops, peak = linear_summary(case, ms, kern, args.steps, pk, pk_kind)
+        out["tflops"] = tflops
+        out["roofline"] = linear_roofline(case, kern, args.steps, pk, pk_kind)
+    out["gpu_launches"] = int(launches)
+    out["clocks"] = clocks.summary()
+
+    if not args.no_e2e:
+        k = max(1, min(args.steps, 10))
+        e_ms = dist.max(time_e2e(case, dist, k))
+        out["e2e"] = {"value": dist.sum(case.tokens * k) / (e_ms * 1e-3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": case.h2d, "d2h_bytes_per_step": case.d2h,
+                      "path": "pinned host -> device copies, gh C ABI call, loss read back, per step"}
+
+    if is_ce and not args.no_linear and dist.world >= 1:
+        try:
+            lcase = LinearCase("linear_ce_gpt2", dist.rank, dev)
+            lsteps = max(3, min(args.steps, 20))
+            lms, llaunch, lkern = time_steps(lcase, dist, lsteps, args.warmup, None)
+            lms = dist.max(lms)
+            tot_ms, tflops, gemm_ms, gemm_tflops, peak = linear_summary(lcase, lms, lkern, lsteps, pk, pk_kind)
+            out["linear_ce"] = {"workload": lcase.p.name, "value": dist.sum(lcase.tokens * lsteps) / (lms * 1e-3),
+                                "unit": "tokens/s", "ms_per_step": lms / lsteps, "tflops": tflops,
+                                "steps": lsteps, "gpu_launches": int(llaunch),
+                                "roofline": linear_roofline(lcase, lkern, lsteps, pk, pk_kind)}
+            del lcase
+        except Exception as e:  # the CE line stands on its own
+            out["linear_ce"] = {"unavailable": f"{type(e).__name__}: {e}"}
+
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        rows = ORACLE_ROWS[args.workload]
+        v, nrows, dt = run_oracle_timing(case, rows)
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1 if is_ce else cpu_threads(),
+                               "kind": "oracle",
+                               "sample": f"first {nrows} rows of the same workload, float64 numpy oracle, "
+                                         f"{dt:.1f} s"}
+    if dist.rank == 0:
+        print(json.dumps(out), flush=True)
+    dist.close()
+
+
+def linear_roofline(case, kern, steps, pk, pk_kind):
+    peak = pk.get("bf16_tflops_sustained") or pk.get("bf16_tflops")
+    gemm_ms = sum(kern[k][0] for k in ("logits_gemm", "dx_gemm", "dw_gemm")) / steps
+    per = {k: kern[k][0] / max(kern[k][1], 1) for k in kern}
+    achieved = case.flops_per_step / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    return {"bound": "tensor", "kernel": "tcgen05 GEMMs (logits, dX, dW) per step",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": (achieved / peak) if achieved else None, "traffic": None,
+            "algorithmic_flops": case.flops_per_step, "kernel_ms_per_launch": per,
+            "peak_source": f"{pk_kind} bf16 (sustained)"}
+
+
+def reference_arm(args, dist):
+    """The float64 oracle on the host cores, on a bounded sample of the same workload."""
+    if dist.rank != 0:
+        return 0
+    is_ce = args.workload in CE_WORKLOADS
+
+    class Dummy:
+        pass
+    if is_ce:
+        case = Dummy()
+        case.p = make_ce(args.workload, 0)
+        case.kind = "ce"
+        case.cpu_sample = lambda n, c=case: __import__("numpy").arange(min(c.p.B, n))
+        case.run_oracle = lambda rows, c=case: CeCase.run_oracle(c, rows)
+    else:
+        case = Dummy()
+        case.p = make_linear(args.workload, 0)
+        case.kind = "linear"
+        case.cpu_sample = lambda n, c=case: __import__("numpy").arange(min(c.p.N, n))
+        case.run_oracle = lambda rows, c=case: LinearCase.run_oracle(c, rows)
+    rows_per_step = max(1, ORACLE_ROWS[args.workload] // 8)
+    rows = case.cpu_sample(rows_per_step)
+    for _ in range(args.warmup):
+        case.run_oracle(rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        case.run_oracle(rows)
+    dt = time.perf_counter() - t0
+    value = len(rows) * args.steps / dt
+    cores = 1 if is_ce else cpu_threads()
+    sample = f"first {len(rows)} rows of {case.p.name} per step, float64 numpy oracle"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64", "data": "synthetic (seeded)", "config": {"workload": case.p.name},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

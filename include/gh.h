@@ -1,0 +1,171 @@
+/*
+ * gh.h — C ABI of libgh, next-token cross-entropy for NVIDIA B200 (sm_100a).
+ *
+ * Two operations, both from the Greyhound functional API
+ * (greyhound.nn.functional):
+ *
+ *  - gh_ce_fwd_bwd: `cross_entropy` — materialised [B, V] logits and [B]
+ *    targets; the summed (or mean) loss with optional z-loss and the logits
+ *    gradient "in one streaming pass".  nuvec FastOp::CrossEntropy gives the
+ *    row loss logsumexp(x) - x[target] (float32) and FastOp::CrossEntropyVjp
+ *    its logits gradient.
+ *  - gh_linear_ce: `chunked_linear_cross_entropy` — logits = inputs @ weight.T
+ *    computed one row chunk at a time and never materialised in full; per
+ *    chunk the logits gradient G gives grad_inputs[chunk] = G @ weight and
+ *    grad_weight += G.T @ inputs[chunk] (`chunked_linear_loss`), with the
+ *    weight-gradient accumulator in fp32 or in the weight dtype
+ *    (`grad_weight_accum_dtype`).
+ *
+ * Definitions (x = one logits row, t its target, ii = ignore_index,
+ * z = z-loss multiplier, lse = log sum_j exp(x_j)):
+ *     row loss  = (lse - x_t) + z * lse^2          if t != ii, else 0
+ *     grad_j    = scale * ((1 + 2 z lse) * exp(x_j - lse) - [j == t])
+ *     scale     = 1 / max(n_valid, 1) for GH_REDUCTION_MEAN, 1 for SUM
+ *     loss      = sum of row losses * (1 / max(n_valid, 1) for MEAN)
+ * where n_valid counts the targets that are not ii (over the whole call; in
+ * linear-CE over all N rows, not per chunk).  Rows whose target equals ii
+ * contribute no loss and an all-zero gradient row.  Gradients are those of the
+ * returned loss (upstream gradient 1).
+ *
+ * Common rules for every entry point:
+ *  - Tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *    contiguous (row stride = number of columns).  The library keeps no
+ *    pointer after the call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Work is enqueued on it and the call returns without waiting;
+ *    outputs are valid once the stream reaches that point.  The library
+ *    allocates its scratch stream-ordered (cudaMallocAsync/cudaFreeAsync) on
+ *    the same stream.
+ *  - Arguments are validated on the host before anything is enqueued:
+ *    null pointers, negative sizes, unknown enums and non-finite z give
+ *    GH_ERR_INVALID_ARG and nothing runs.  B == 0 (or N == 0) writes loss = 0.
+ *  - A target outside [0, V) that is not ii violates the precondition; it
+ *    cannot be seen on the host without a sync, so the kernels treat that row
+ *    as ignored (no out-of-bounds access) and record GH_ERR_TARGET_RANGE in
+ *    the device status word (read it with gh_get_device_status).
+ *  - Every device-side wait is bounded; a wait that runs out records
+ *    GH_ERR_TIMEOUT in the status word and the kernel returns.
+ *  - The library is not thread-safe across concurrent calls that share a
+ *    stream only in the sense CUDA streams are; distinct streams are fine.
+ */
+#ifndef GH_H_
+#define GH_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GH_OK = 0,
+  GH_ERR_INVALID_ARG = 1,  /* rejected on the host; nothing was enqueued */
+  GH_ERR_UNSUPPORTED = 2,  /* valid request outside what this build supports */
+  GH_ERR_ALLOC = 3,        /* scratch allocation failed; nothing was enqueued */
+  GH_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed */
+  GH_ERR_TIMEOUT = 5,      /* a bounded device wait ran out (device status) */
+  GH_ERR_TARGET_RANGE = 6  /* a target outside [0, V) was seen (device status) */
+} gh_status_t;
+
+/* Greyhound `reduction`: "mean" divides the summed loss by the number of
+ * valid tokens, "sum" returns the summed loss. */
+typedef enum { GH_REDUCTION_MEAN = 0, GH_REDUCTION_SUM = 1 } gh_reduction_t;
+
+/* Greyhound `grad_weight_accum_dtype`: "fp32" accumulates the per-chunk
+ * weight-gradient products in fp32 and casts once at the end; "weight"
+ * accumulates in the weight dtype, rounding between chunks. */
+typedef enum { GH_ACCUM_FP32 = 0, GH_ACCUM_WEIGHT = 1 } gh_accum_t;
+
+/* Element type of logits / gradients. */
+typedef enum { GH_F32 = 0, GH_BF16 = 1 } gh_dtype_t;
+
+/*
+ * gh_ce_fwd_bwd — standalone cross-entropy, forward and backward in one call
+ * (Greyhound `cross_entropy`).
+ *
+ *   logits   [B, V] of `dtype` (GH_F32 or GH_BF16), device.
+ *   targets  [B] int64 class ids, device.
+ *   B >= 0, V >= 1 (V < 2^31).
+ *   ignore_index  target value that is ignored (may lie inside [0, V)).
+ *   reduction     GH_REDUCTION_MEAN or GH_REDUCTION_SUM.
+ *   z_mult        z-loss multiplier (finite; 0 disables).
+ *   loss     device float32 scalar, written.
+ *   grad     [B, V] of `dtype`, device, written with the logits gradient
+ *            (round to nearest even).  grad == logits is allowed (in place,
+ *            as the raw kernel helper on the Greyhound page does); any other
+ *            overlap is not.
+ *   stream   cudaStream_t as void*.
+ */
+gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B, int64_t V,
+                          gh_dtype_t dtype, int64_t ignore_index, gh_reduction_t reduction,
+                          float z_mult, float* loss, void* grad, void* stream);
+
+/*
+ * gh_linear_ce — chunked fused linear cross-entropy (Greyhound
+ * `chunked_linear_cross_entropy` over `chunked_linear_loss`).
+ *
+ *   inputs       [N, D] bf16, device (hidden states, one row per token).
+ *   weight       [V, D] bf16, device (LM head; logits = inputs @ weight.T).
+ *   targets      [N] int64, device.
+ *   N >= 0, D >= 1, V >= 1; D must be a multiple of 8 (16-byte rows for TMA).
+ *   chunk        rows per logits chunk; <= 0 selects the default (the largest
+ *                multiple of 128 whose bf16 chunk logits fit 1 GiB, capped at N).
+ *   accum_dtype  GH_ACCUM_FP32 or GH_ACCUM_WEIGHT.
+ *   ignore_index, reduction, z_mult  as for gh_ce_fwd_bwd.
+ *   loss         device float32 scalar, written.
+ *   grad_inputs  [N, D] bf16, device, written.
+ *   grad_weight  [V, D] bf16, device, written (overwritten, not added to).
+ *   stream       cudaStream_t as void*.
+ * Scratch (stream-ordered): chunk x round_up(V, 8) bf16 logits/gradient,
+ * an fp32 [V, D] accumulator when accum_dtype == GH_ACCUM_FP32, and O(N) floats.
+ */
+gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* targets,
+                         int64_t N, int64_t D, int64_t V, int64_t chunk, gh_accum_t accum_dtype,
+                         int64_t ignore_index, gh_reduction_t reduction, float z_mult,
+                         float* loss, void* grad_inputs, void* grad_weight, void* stream);
+
+/*
+ * gh_get_device_status — synchronises `stream`, returns the first error any
+ * kernel recorded on the current device since the last call (GH_OK if none:
+ * GH_ERR_TARGET_RANGE or GH_ERR_TIMEOUT), and clears it.  Returns GH_ERR_CUDA
+ * if the synchronisation itself fails.
+ */
+gh_status_t gh_get_device_status(void* stream);
+
+/*
+ * Kernel timing (for benchmarks and roofline reports).  Kernel kinds: */
+typedef enum {
+  GH_KERNEL_CE_ROW = 0,        /* standalone CE row kernel (one per gh_ce_fwd_bwd) */
+  GH_KERNEL_LOGITS_GEMM = 1,   /* linear-CE: chunk logits = X_c @ W^T (+ CE epilogue) */
+  GH_KERNEL_CHUNK_CE = 2,      /* linear-CE: per-chunk loss and logits gradient */
+  GH_KERNEL_DX_GEMM = 3,       /* linear-CE: grad_inputs[chunk] = G_c @ W */
+  GH_KERNEL_DW_GEMM = 4,       /* linear-CE: grad_weight (+)= G_c^T @ X_c */
+  GH_KERNEL_KINDS = 5
+} gh_kernel_t;
+
+/* gh_profile_enable(1) discards earlier records and starts recording a pair
+ * of CUDA events around every launch of the kernels above, on the launching
+ * stream; gh_profile_enable(0) stops recording (records are kept). */
+gh_status_t gh_profile_enable(int enable);
+
+/* Waits for the recorded events of `kind` and returns their summed elapsed
+ * milliseconds and the number of launches recorded.  Either output may be
+ * NULL.  Returns GH_ERR_INVALID_ARG for an unknown kind, GH_ERR_CUDA if an
+ * event query fails. */
+gh_status_t gh_profile_read(gh_kernel_t kind, double* total_ms, int64_t* launches);
+
+/* Number of kernels this library has launched in this process (all kinds,
+ * including the small counting/reduction kernels). */
+int64_t gh_launch_count(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char* gh_status_string(gh_status_t status);
+
+/* Library version string, e.g. "gh 0.1.0 sm_100a". */
+const char* gh_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GH_H_ */

@@ -1,0 +1,218 @@
+"""B200-native next-token cross-entropy: Python binding of ``libgh.so``.
+
+The functions here only marshal arguments into the C ABI declared in
+``include/gh.h``; every step of the computation runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  There is no
+CPU or PyTorch fallback: if ``libgh.so`` is missing or a call fails, an
+exception is raised.
+
+* ``gh_ce_fwd_bwd`` — Greyhound ``cross_entropy``: loss and logits gradient of
+  materialised ``[B, V]`` logits in one call.
+* ``gh_linear_ce`` — Greyhound ``chunked_linear_cross_entropy``: loss,
+  ``grad_inputs`` and ``grad_weight`` of ``inputs @ weight.T`` computed chunk
+  by chunk, without the full logits.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgh.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gh.h")
+
+GH_OK = 0
+GH_ERR_INVALID_ARG = 1
+GH_ERR_UNSUPPORTED = 2
+GH_ERR_ALLOC = 3
+GH_ERR_CUDA = 4
+GH_ERR_TIMEOUT = 5
+GH_ERR_TARGET_RANGE = 6
+
+GH_REDUCTION = {"mean": 0, "sum": 1}
+GH_ACCUM = {"fp32": 0, "weight": 1}
+GH_F32, GH_BF16 = 0, 1
+
+
+class GhError(RuntimeError):
+    """A libgh call returned a status other than GH_OK."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libgh.so`` with argument types set (loads on first use)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m lm_head_cross_gh_b200._build` "
+            "(nvcc, sm_100a).  There is no fallback implementation.")
+    L = ctypes.CDLL(LIB_PATH)
+    c_void_p, c_int64, c_int, c_float = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    L.gh_ce_fwd_bwd.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_int, c_float,
+                                c_void_p, c_void_p, c_void_p]
+    L.gh_ce_fwd_bwd.restype = c_int
+    L.gh_linear_ce.argtypes = [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int,
+                               c_int64, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p]
+    L.gh_linear_ce.restype = c_int
+    L.gh_get_device_status.argtypes = [c_void_p]
+    L.gh_get_device_status.restype = c_int
+    L.gh_status_string.argtypes = [c_int]
+    L.gh_status_string.restype = ctypes.c_char_p
+    L.gh_version.argtypes = []
+    L.gh_version.restype = ctypes.c_char_p
+    L.gh_profile_enable.argtypes = [c_int]
+    L.gh_profile_enable.restype = c_int
+    L.gh_profile_read.argtypes = [c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_int64)]
+    L.gh_profile_read.restype = c_int
+    L.gh_launch_count.argtypes = []
+    L.gh_launch_count.restype = c_int64
+    _lib = L
+    return L
+
+
+def header_symbols() -> list:
+    """Names of the functions ``include/gh.h`` declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gh_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib().gh_status_string(int(status)).decode()
+
+
+def gh_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def gh_version() -> str:
+    return lib().gh_version().decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != GH_OK:
+        raise GhError(status, where)
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _need(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+def gh_ce_fwd_bwd(logits, targets, ignore_index: int = -100, reduction: str = "mean",
+                  z_loss: float = 0.0, *, grad=None, loss=None, stream=None):
+    """Cross-entropy loss and logits gradient (one call into ``gh_ce_fwd_bwd``).
+
+    ``logits``: CUDA tensor [B, V], float32 or bfloat16, contiguous.
+    ``targets``: CUDA int64 [B].  ``grad`` (optional output, same shape and
+    dtype; may be ``logits`` itself for the in-place form) and ``loss``
+    (optional float32 scalar output) are allocated when not given.
+    Returns ``(loss, grad)``; both are valid on ``stream`` when the call returns.
+    """
+    import torch
+    _need(logits.dim() == 2 and logits.is_cuda and logits.is_contiguous(), "logits: contiguous CUDA [B, V]")
+    _need(logits.dtype in (torch.float32, torch.bfloat16), "logits dtype must be float32 or bfloat16")
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
+          and targets.shape == (logits.shape[0],), "targets: contiguous CUDA int64 [B]")
+    _need(reduction in GH_REDUCTION, "reduction must be 'mean' or 'sum'")
+    if grad is None:
+        grad = torch.empty_like(logits)
+    _need(grad.shape == logits.shape and grad.dtype == logits.dtype and grad.is_contiguous(), "grad mismatch")
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=logits.device)
+    _need(loss.dtype == torch.float32 and loss.numel() == 1, "loss must be a float32 scalar")
+    B, V = logits.shape
+    dtype = GH_F32 if logits.dtype == torch.float32 else GH_BF16
+    st = lib().gh_ce_fwd_bwd(_ptr(logits), _ptr(targets), B, V, dtype, int(ignore_index),
+                             GH_REDUCTION[reduction], float(z_loss), _ptr(loss), _ptr(grad),
+                             _stream_handle(stream))
+    _check(st, "gh_ce_fwd_bwd")
+    return loss, grad
+
+
+def gh_linear_ce(inputs, weight, targets, ignore_index: int = -100, reduction: str = "mean",
+                 z_loss: float = 0.0, chunk: int = 0, accum: str = "fp32", *, grad_inputs=None,
+                 grad_weight=None, loss=None, stream=None):
+    """Chunked linear cross-entropy (one call into ``gh_linear_ce``).
+
+    ``inputs`` bf16 [N, D], ``weight`` bf16 [V, D], ``targets`` int64 [N], all
+    contiguous CUDA tensors.  ``chunk`` rows per logits chunk (<= 0: default),
+    ``accum`` "fp32" or "weight".  Returns ``(loss, grad_inputs, grad_weight)``.
+    """
+    import torch
+    _need(inputs.dim() == 2 and weight.dim() == 2 and inputs.shape[1] == weight.shape[1], "shapes")
+    _need(inputs.dtype == torch.bfloat16 and weight.dtype == torch.bfloat16, "inputs/weight must be bfloat16")
+    _need(inputs.is_cuda and weight.is_cuda and inputs.is_contiguous() and weight.is_contiguous(), "layout")
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
+          and targets.shape == (inputs.shape[0],), "targets: contiguous CUDA int64 [N]")
+    _need(reduction in GH_REDUCTION and accum in GH_ACCUM, "reduction / accum")
+    if grad_inputs is None:
+        grad_inputs = torch.empty_like(inputs)
+    if grad_weight is None:
+        grad_weight = torch.empty_like(weight)
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=inputs.device)
+    N, D = inputs.shape
+    V = weight.shape[0]
+    st = lib().gh_linear_ce(_ptr(inputs), _ptr(weight), _ptr(targets), N, D, V, int(chunk), GH_ACCUM[accum],
+                            int(ignore_index), GH_REDUCTION[reduction], float(z_loss), _ptr(loss),
+                            _ptr(grad_inputs), _ptr(grad_weight), _stream_handle(stream))
+    _check(st, "gh_linear_ce")
+    return loss, grad_inputs, grad_weight
+
+
+GH_KERNEL = {"ce_row": 0, "logits_gemm": 1, "chunk_ce": 2, "dx_gemm": 3, "dw_gemm": 4}
+
+
+def gh_profile_enable(enable: bool = True) -> None:
+    """Start (discarding earlier records) or stop recording per-kernel CUDA events."""
+    _check(lib().gh_profile_enable(1 if enable else 0), "gh_profile_enable")
+
+
+def gh_profile_read(kind: str):
+    """(summed milliseconds, launches) recorded for one kernel kind."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int64(0)
+    _check(lib().gh_profile_read(GH_KERNEL[kind], ctypes.byref(ms), ctypes.byref(n)), "gh_profile_read")
+    return ms.value, n.value
+
+
+def gh_launch_count() -> int:
+    """Kernels launched by libgh in this process so far."""
+    return int(lib().gh_launch_count())
+
+
+def gh_get_device_status(stream=None) -> int:
+    """Synchronise ``stream``; return and clear the device status word."""
+    return int(lib().gh_get_device_status(_stream_handle(stream)))
+
+
+__all__ = [
+    "GhError", "lib", "header_symbols", "status_string", "gh_status_string", "gh_version",
+    "gh_ce_fwd_bwd", "gh_linear_ce", "gh_get_device_status", "gh_profile_enable", "gh_profile_read",
+    "gh_launch_count", "GH_KERNEL",
+    "GH_OK", "GH_ERR_INVALID_ARG", "GH_ERR_UNSUPPORTED", "GH_ERR_ALLOC", "GH_ERR_CUDA",
+    "GH_ERR_TIMEOUT", "GH_ERR_TARGET_RANGE", "GH_REDUCTION", "GH_ACCUM", "GH_F32", "GH_BF16",
+]

@@ -1,0 +1,187 @@
+// C ABI of libgh (declared in include/gh.h): host-side validation, scratch
+// management and dispatch to the kernels.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+
+#include "ce.h"
+#include "common.cuh"
+#include "linear_ce.h"
+#include "profile.h"
+
+namespace gh {
+
+// Scratch is stream-ordered.  GH_FAULT_ALLOC=1 makes every scratch allocation
+// fail (host-side fault injection for the error path; nothing is enqueued).
+static bool fault_alloc() {
+  const char* e = std::getenv("GH_FAULT_ALLOC");
+  return e && e[0] == '1';
+}
+
+gh_status_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
+  *p = nullptr;
+  if (fault_alloc()) return GH_ERR_ALLOC;
+  if (bytes == 0) bytes = 16;
+  if (cudaMallocAsync(p, bytes, stream) != cudaSuccess) {
+    (void)cudaGetLastError();
+    *p = nullptr;
+    return GH_ERR_ALLOC;
+  }
+  return GH_OK;
+}
+
+void scratch_free(void* p, cudaStream_t stream) {
+  if (p) (void)cudaFreeAsync(p, stream);
+}
+
+}  // namespace gh
+
+using namespace gh;
+
+extern "C" {
+
+gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B, int64_t V, gh_dtype_t dtype,
+                          int64_t ignore_index, gh_reduction_t reduction, float z_mult, float* loss, void* grad,
+                          void* stream_) {
+  if (B < 0 || V < 1 || V >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
+  if (dtype != GH_F32 && dtype != GH_BF16) return GH_ERR_INVALID_ARG;
+  if (reduction != GH_REDUCTION_MEAN && reduction != GH_REDUCTION_SUM) return GH_ERR_INVALID_ARG;
+  if (!std::isfinite(z_mult)) return GH_ERR_INVALID_ARG;
+  if (!loss) return GH_ERR_INVALID_ARG;
+  if (B > 0 && (!logits || !targets || !grad)) return GH_ERR_INVALID_ARG;
+  const int es = dtype == GH_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(logits) % es) || (reinterpret_cast<uintptr_t>(grad) % es) ||
+      (reinterpret_cast<uintptr_t>(targets) % 8) || (reinterpret_cast<uintptr_t>(loss) % 4))
+    return GH_ERR_INVALID_ARG;
+  if (grad != logits && B > 0) {
+    // Partial overlap of grad and logits is not allowed (exact aliasing is).
+    const uintptr_t l0 = reinterpret_cast<uintptr_t>(logits), g0 = reinterpret_cast<uintptr_t>(grad);
+    const uintptr_t bytes = static_cast<uintptr_t>(B) * static_cast<uintptr_t>(V) * es;
+    if (l0 < g0 + bytes && g0 < l0 + bytes) return GH_ERR_INVALID_ARG;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (B == 0) return cudaMemsetAsync(loss, 0, sizeof(float), stream) == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+
+  void* scratch = nullptr;
+  gh_status_t st = scratch_alloc(&scratch, 16 + static_cast<size_t>(B) * sizeof(float), stream);
+  if (st != GH_OK) return st;
+  unsigned long long* n_valid = static_cast<unsigned long long*>(scratch);
+  float* row_loss = reinterpret_cast<float*>(static_cast<char*>(scratch) + 16);
+
+  const int mean = reduction == GH_REDUCTION_MEAN;
+  st = ce_count_launch(targets, B, V, ignore_index, n_valid, stream);
+  if (st == GH_OK) {
+    CeArgs a{};
+    a.logits = logits;
+    a.grad = grad;
+    a.targets = targets;
+    a.V = V;
+    a.ld = V;
+    a.ignore_index = ignore_index;
+    a.z = z_mult;
+    a.mean = mean;
+    a.n_valid = n_valid;
+    a.row_loss = row_loss;
+    a.congruent = ((reinterpret_cast<uintptr_t>(logits) ^ reinterpret_cast<uintptr_t>(grad)) & 15) == 0;
+    st = ce_launch(a, B, dtype, stream);
+  }
+  if (st == GH_OK) st = ce_reduce_launch(row_loss, B, n_valid, mean, loss, stream);
+  scratch_free(scratch, stream);
+  return st;
+}
+
+gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* targets, int64_t N, int64_t D,
+                         int64_t V, int64_t chunk, gh_accum_t accum_dtype, int64_t ignore_index,
+                         gh_reduction_t reduction, float z_mult, float* loss, void* grad_inputs, void* grad_weight,
+                         void* stream_) {
+  if (N < 0 || D < 1 || V < 1 || V >= (int64_t(1) << 31) || D >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
+  if (D % 8) return GH_ERR_INVALID_ARG;
+  if (accum_dtype != GH_ACCUM_FP32 && accum_dtype != GH_ACCUM_WEIGHT) return GH_ERR_INVALID_ARG;
+  if (reduction != GH_REDUCTION_MEAN && reduction != GH_REDUCTION_SUM) return GH_ERR_INVALID_ARG;
+  if (!std::isfinite(z_mult)) return GH_ERR_INVALID_ARG;
+  if (!loss || !weight || !grad_weight) return GH_ERR_INVALID_ARG;
+  if (N > 0 && (!inputs || !targets || !grad_inputs)) return GH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(inputs) % 16) || (reinterpret_cast<uintptr_t>(weight) % 16) ||
+      (reinterpret_cast<uintptr_t>(grad_inputs) % 16) || (reinterpret_cast<uintptr_t>(grad_weight) % 16) ||
+      (reinterpret_cast<uintptr_t>(targets) % 8) || (reinterpret_cast<uintptr_t>(loss) % 4))
+    return GH_ERR_INVALID_ARG;
+  LinearCeArgs a{};
+  a.X = inputs;
+  a.W = weight;
+  a.targets = targets;
+  a.N = N;
+  a.D = D;
+  a.V = V;
+  a.chunk = chunk;
+  a.accum = accum_dtype;
+  a.ignore_index = ignore_index;
+  a.mean = reduction == GH_REDUCTION_MEAN;
+  a.z = z_mult;
+  a.loss = loss;
+  a.dX = grad_inputs;
+  a.dW = grad_weight;
+  return linear_ce_run(a, static_cast<cudaStream_t>(stream_));
+}
+
+gh_status_t gh_get_device_status(void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return GH_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return GH_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return GH_ERR_CUDA;
+  return static_cast<gh_status_t>(v);
+}
+
+gh_status_t gh_profile_enable(int enable) {
+  ProfileState& s = profile_state();
+  std::lock_guard<std::mutex> g(s.mu);
+  if (enable) {
+    for (auto& r : s.recs) {
+      (void)cudaEventSynchronize(r.stop);
+      s.pool.push_back(r.start);
+      s.pool.push_back(r.stop);
+    }
+    s.recs.clear();
+  }
+  s.enabled = enable != 0;
+  return GH_OK;
+}
+
+gh_status_t gh_profile_read(gh_kernel_t kind, double* total_ms, int64_t* launches) {
+  if (kind < 0 || kind >= GH_KERNEL_KINDS) return GH_ERR_INVALID_ARG;
+  ProfileState& s = profile_state();
+  std::lock_guard<std::mutex> g(s.mu);
+  double tot = 0.0;
+  int64_t n = 0;
+  for (auto& r : s.recs) {
+    if (r.kind != kind) continue;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) return GH_ERR_CUDA;
+    float ms = 0.0f;
+    if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) return GH_ERR_CUDA;
+    tot += ms;
+    ++n;
+  }
+  if (total_ms) *total_ms = tot;
+  if (launches) *launches = n;
+  return GH_OK;
+}
+
+int64_t gh_launch_count(void) { return launch_counter().load(); }
+
+const char* gh_status_string(gh_status_t s) {
+  switch (s) {
+    case GH_OK: return "ok";
+    case GH_ERR_INVALID_ARG: return "invalid argument";
+    case GH_ERR_UNSUPPORTED: return "unsupported";
+    case GH_ERR_ALLOC: return "scratch allocation failed";
+    case GH_ERR_CUDA: return "CUDA error";
+    case GH_ERR_TIMEOUT: return "device wait timed out";
+    case GH_ERR_TARGET_RANGE: return "target outside [0, V)";
+  }
+  return "unknown status";
+}
+
+const char* gh_version(void) { return "gh 0.1.0 sm_100a"; }
+
+}  // extern "C"

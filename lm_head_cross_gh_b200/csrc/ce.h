@@ -1,0 +1,41 @@
+// Internal interface of the standalone cross-entropy kernels (ce.cu).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/gh.h"
+
+namespace gh {
+
+struct CeArgs {
+  const void* logits;                 // [B, V] row-major
+  void* grad;                         // [B, V] row-major, same dtype
+  const int64_t* targets;             // [B]
+  int64_t V;
+  int64_t ld;                         // row stride in elements (>= V)
+  int64_t ignore_index;
+  float z;                            // z-loss multiplier
+  int mean;                           // 1: divide by n_valid
+  const unsigned long long* n_valid;  // written by ce_count_kernel
+  float* row_loss;                    // [B] scratch
+  int slice;                          // elements per CTA (set by ce_launch)
+  int cluster;                        // CTAs per row (set by ce_launch)
+  int congruent;                      // (logits - grad) % 16 == 0
+};
+
+struct CePlan {
+  bool streaming;  // row too long for the shared-memory path
+  int cluster;     // CTAs per row
+  int slice;       // elements per CTA
+  int smem_bytes;  // dynamic shared memory per CTA
+};
+
+CePlan ce_plan(int64_t V, int elem_bytes);
+gh_status_t ce_count_launch(const int64_t* targets, int64_t n, int64_t V, int64_t ii,
+                            unsigned long long* count, cudaStream_t stream);
+gh_status_t ce_launch(const CeArgs& args, int64_t B, gh_dtype_t dtype, cudaStream_t stream);
+gh_status_t ce_reduce_launch(const float* row_loss, int64_t B, const unsigned long long* n_valid, int mean,
+                             float* loss, cudaStream_t stream);
+
+}  // namespace gh

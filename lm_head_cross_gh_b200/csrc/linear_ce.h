@@ -1,0 +1,31 @@
+// Internal interface of the chunked linear cross-entropy (linear_ce.cu).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/gh.h"
+
+namespace gh {
+
+struct LinearCeArgs {
+  const void* X;           // [N, D] bf16
+  const void* W;           // [V, D] bf16
+  const int64_t* targets;  // [N]
+  int64_t N, D, V;
+  int64_t chunk;           // <= 0: default
+  gh_accum_t accum;
+  int64_t ignore_index;
+  int mean;
+  float z;
+  float* loss;             // device scalar
+  void* dX;                // [N, D] bf16
+  void* dW;                // [V, D] bf16
+};
+
+gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream);
+
+gh_status_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream);
+void scratch_free(void* p, cudaStream_t stream);
+
+}  // namespace gh
