@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "ce.h"
 #include "common.cuh"
@@ -11,18 +12,48 @@
 
 namespace gh {
 
-// Scratch is stream-ordered.  GH_FAULT_ALLOC=1 makes every scratch allocation
-// fail (host-side fault injection for the error path; nothing is enqueued).
+// Scratch is stream-ordered, from a memory pool the library creates per
+// device.  The pool keeps freed memory (release threshold: 4 GiB) so calls do
+// not return memory to the driver and map it again every time.
+// GH_FAULT_ALLOC=1 makes every scratch allocation fail (host-side fault
+// injection for the error path; nothing is enqueued).
 static bool fault_alloc() {
   const char* e = std::getenv("GH_FAULT_ALLOC");
   return e && e[0] == '1';
+}
+
+static std::mutex g_pool_mu;
+static cudaMemPool_t g_pools[64] = {};
+
+static cudaMemPool_t device_pool(int dev) {
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> g(g_pool_mu);
+  if (!g_pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    uint64_t keep = 4ull << 30;
+    (void)cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    g_pools[dev] = pool;
+  }
+  return g_pools[dev];
 }
 
 gh_status_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
   *p = nullptr;
   if (fault_alloc()) return GH_ERR_ALLOC;
   if (bytes == 0) bytes = 16;
-  if (cudaMallocAsync(p, bytes, stream) != cudaSuccess) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GH_ERR_CUDA;
+  cudaMemPool_t pool = device_pool(dev);
+  const cudaError_t e = pool ? cudaMallocFromPoolAsync(p, bytes, pool, stream) : cudaMallocAsync(p, bytes, stream);
+  if (e != cudaSuccess) {
     (void)cudaGetLastError();
     *p = nullptr;
     return GH_ERR_ALLOC;

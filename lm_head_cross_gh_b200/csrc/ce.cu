@@ -5,14 +5,15 @@
 //
 // Kernels, in launch order on the caller's stream:
 //   ce_count_kernel  n_valid = #{t != ignore_index}; flags targets outside [0, V)
-//   ce_row_kernel    one CTA (or a cluster of S CTAs) per row.  Each CTA pulls
-//                    its slice of the row into shared memory with one bulk
-//                    async copy per piece, folds an online (max, sum-exp) over
-//                    it as the pieces land, exchanges the partial (max, sum)
-//                    with its cluster peers through distributed shared memory,
-//                    then rewrites the slice in place as the gradient and
-//                    streams it back with a bulk async store.  HBM sees one
-//                    read and one write of every logit.
+//   ce_row_kernel    persistent; one CTA (or a cluster of S CTAs) per row at a
+//                    time.  Each CTA pulls its slice of a row into one of two
+//                    shared-memory buffers with a bulk async copy (the next
+//                    rows' copies are in flight while a row is computed), takes
+//                    the max, caches exp(x - max) once per element, exchanges
+//                    partial (max, sum) with its cluster peers through
+//                    distributed shared memory, and stores the gradient
+//                    straight to global.  HBM sees one read and one write of
+//                    every logit.
 //   ce_stream_kernel rows too long for the cluster path: two passes over
 //                    global memory (the second one mostly from L2).
 //   ce_reduce_kernel fixed-order (deterministic) sum of the per-row losses,
@@ -21,6 +22,7 @@
 #include <climits>
 #include <cstdio>
 #include <cstdlib>
+#include <mutex>
 
 #include "ce.h"
 #include "common.cuh"
@@ -211,6 +213,12 @@ __device__ __forceinline__ float2 f16x2_to_f32(uint32_t w) {
   return make_float2(lo, hi);
 }
 
+__device__ __forceinline__ float f16_to_f32(uint16_t h) {
+  float f;
+  asm("{\n\t.reg .f16 x;\n\tmov.b16 x, %1;\n\tcvt.f32.f16 %0, x;\n\t}" : "=f"(f) : "h"(h));
+  return f;
+}
+
 template <int N>
 __device__ __forceinline__ void unpack_f16x8(const uint4& q, float (&g)[N]) {
   const float2 a = f16x2_to_f32(q.x), b = f16x2_to_f32(q.y), c = f16x2_to_f32(q.z), d = f16x2_to_f32(q.w);
@@ -218,23 +226,82 @@ __device__ __forceinline__ void unpack_f16x8(const uint4& q, float (&g)[N]) {
   if constexpr (N == 8) { g[4] = c.x; g[5] = c.y; g[6] = d.x; g[7] = d.y; }
 }
 
-constexpr int kMaxPieces = 4;
-constexpr int kMinPieceChunks = 256;  // 4 KiB
-constexpr int kRowThreads = 256;
+constexpr int kRowThreads = 512;
 constexpr int kStreamThreads = 1024;
-constexpr int kHdrBytes = 128;        // barriers, cluster record, reduction scratch
+constexpr int kPieces = 4;                     // bulk copies (and barriers) per slice
+constexpr int kMinPieceChunks = 256;           // 4 KiB
+constexpr int kHdrBytes = 384;                 // barriers, targets, records, reduction scratch
+constexpr int kMaxSliceBytes = 110 * 1024;     // two slice buffers per CTA fit in 227 KiB
 
 struct RowShared {
-  uint64_t bars[kMaxPieces];  // 32 B
-  float rec_m, rec_s, rec_xt;  // partial published to the cluster
-  int rec_has_t;
-  float lse, xt;               // broadcast after the exchange
-  float xt_local;              // target logit, when it lies in this CTA's slice
-  float pad_;
+  uint64_t full[2][kPieces];                   // load barriers of the two buffer slots
+  int64_t tgt[2][2];                           // per group: targets of its next two rows
+  float rec_m[2], rec_s[2], rec_xt[2];         // partials published to the cluster,
+  int rec_has_t[2];                            //   double-buffered by valid-row parity
+  float lse[2], xt[2], xt_local[2];            // per group, broadcast within the group
+  float pad_[2];
   float red_m[kRowThreads / 32];
   float red_s[kRowThreads / 32];
 };
 static_assert(sizeof(RowShared) <= kHdrBytes, "header too large");
+
+// Geometry of one CTA's slice of one row: elements [e0, e0 + n) at global
+// address gsrc.  Slice buffer byte j <-> global byte (gsrc - lead + j).
+// Chunks [c_lo, c_hi) are whole 16-byte chunks inside the slice; the chunks
+// before and after hold the ragged ends.  Chunks [x_lo, x_hi) are copied in
+// bulk: the ragged-end chunks too, whenever their 16 bytes lie inside the
+// logits buffer (the bytes outside the slice are then overwritten with -inf).
+struct SliceGeo {
+  const uint8_t* gsrc;
+  uint8_t* gdst;
+  int n, lead, span, nchunks, c_lo, c_hi, x_lo, x_hi;
+};
+
+template <int ES>
+__device__ __forceinline__ SliceGeo slice_geo(const CeArgs& a, int64_t row, int rank) {
+  SliceGeo g;
+  const int64_t e0 = static_cast<int64_t>(rank) * a.slice;
+  g.n = static_cast<int>(tmax<int64_t>(0, tmin<int64_t>(a.V, e0 + a.slice) - e0));
+  g.gsrc = reinterpret_cast<const uint8_t*>(a.logits) + (row * a.ld + e0) * ES;
+  g.gdst = reinterpret_cast<uint8_t*>(a.grad) + (row * a.ld + e0) * ES;
+  g.lead = static_cast<int>(reinterpret_cast<uintptr_t>(g.gsrc) & 15);
+  g.span = g.lead + g.n * ES;
+  g.nchunks = (g.span + 15) >> 4;
+  g.c_lo = (g.lead + 15) >> 4;
+  g.c_hi = max(g.c_lo, g.span >> 4);
+  const uint8_t* lo_bound = reinterpret_cast<const uint8_t*>(a.logits);
+  const uint8_t* hi_bound = lo_bound + a.B * a.ld * ES;
+  const uint8_t* gbase = g.gsrc - g.lead;
+  g.x_lo = (g.n > 0 && gbase >= lo_bound) ? 0 : g.c_lo;
+  g.x_hi = (g.n > 0 && gbase + 16 * g.nchunks <= hi_bound) ? g.nchunks : g.c_hi;
+  if (g.x_hi < g.x_lo) g.x_hi = g.x_lo;
+  return g;
+}
+
+__device__ __forceinline__ bool target_valid(const CeArgs& a, int64_t t) {
+  return (t != a.ignore_index) && t >= 0 && t < a.V;
+}
+
+__device__ __forceinline__ int npieces_of(int nbulk) {
+  return nbulk == 0 ? 0 : max(1, min(kPieces, nbulk / kMinPieceChunks));
+}
+
+// Group leader: start the bulk copies of this CTA's slice of `row` into `buf`
+// (one per piece, each on its own barrier).
+template <int ES>
+__device__ __forceinline__ void issue_slice(const CeArgs& a, int64_t row, int64_t t, int rank, uint8_t* buf,
+                                            uint64_t* bars) {
+  if (row >= a.B || !target_valid(a, t)) return;
+  const SliceGeo g = slice_geo<ES>(a, row, rank);
+  const int nb = g.x_hi - g.x_lo;
+  const int np = npieces_of(nb);
+  const uint8_t* gbase = g.gsrc - g.lead;
+  for (int p = 0; p < np; ++p) {
+    const int cs = g.x_lo + (nb * p) / np, ce = g.x_lo + (nb * (p + 1)) / np;
+    mbar_arrive_expect_tx(&bars[p], 16u * (ce - cs));
+    bulk_g2s(buf + 16 * cs, gbase + 16 * cs, 16u * (ce - cs), &bars[p]);
+  }
+}
 
 }  // namespace
 
@@ -255,227 +322,381 @@ __global__ void ce_count_kernel(const int64_t* __restrict__ t, int64_t n, int64_
   if (bad) record_status(GH_ERR_TARGET_RANGE);
 }
 
-// One CTA per slice of `slice` elements; `cluster` CTAs per row (the launch's
-// cluster dimension).  Dynamic shared memory: kHdrBytes + 16 * (chunks + 1).
+// Single-CTA count for batches up to 2^20 rows: no atomics, no prior memset.
+__global__ void __launch_bounds__(1024) ce_count1_kernel(const int64_t* __restrict__ t, int64_t n, int64_t V,
+                                                         int64_t ii, unsigned long long* __restrict__ count) {
+  __shared__ unsigned long long part[32];
+  unsigned long long c = 0;
+  bool bad = false;
+  for (int64_t i = threadIdx.x; i < n; i += 1024) {
+    const int64_t v = t[i];
+    if (v != ii) {
+      if (v >= 0 && v < V) ++c;
+      else bad = true;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+  if (bad) record_status(GH_ERR_TARGET_RANGE);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long tot = 0;
+    for (int w = 0; w < 32; ++w) tot += part[w];
+    *count = tot;
+  }
+}
+
+// Persistent row kernel.  A CTA holds NG independent row groups of
+// kRowThreads / NG threads.  With NG = 2 (rows of one slice) each group owns
+// one slice buffer and its own rows; the two groups drift out of phase, so one
+// group's exponent pass overlaps the other's loads and stores.  With NG = 1 a
+// cluster of `cluster` CTAs shares each row (one slice each) and every CTA
+// double-buffers its slices.  A buffer's bulk copy is split into pieces with
+// one barrier each, so work starts as soon as the first piece lands.
 //
-// Chunk c of the slice buffer (16 bytes) is owned by thread c % kRowThreads in
-// every pass, so the passes need no barrier between them apart from the two
-// block reductions.  Passes, for a bf16 row:
-//   0  max over the slice on packed bf16 pairs, piece by piece as copies land
-//   1  e = 2^14 * exp(x - m) once per element: summed in fp32 and cached in
+// Chunk c (16 bytes) of a slice belongs to thread c % (group size) in every
+// pass, so the passes of a row need no barrier between them; each thread works
+// relative to the max m_t of its own chunks.  For a bf16 row:
+//   0  m_t = max over the thread's chunks, on packed bf16 pairs
+//   1  e = 2^14 exp(x - m_t) once per element: summed in fp32 and cached in
 //      place as fp16 (the 2^14 keeps the cache in fp16's normal range down to
-//      exp(x - m) = 2^-28)
-//   2  gradient = k * e with one per-CTA factor k, stored straight to global
-// For fp32 rows pass 1 only sums and pass 2 re-evaluates the exponent (the
+//      exp(x - m_t) = 2^-28)
+//   *  one group combine of (m_t, s_t); the CTAs of a cluster exchange (max,
+//      sum, target logit) once through distributed shared memory
+//   2  gradient = k_t e, k_t = scale (1 + 2 z lse) 2^-14 exp(m_t - lse),
+//      stored straight to global; the target element is rewritten by its
+//      owner afterwards with the -scale term.
+// fp32 rows only sum in pass 1 and re-evaluate the exponent in pass 2 (a
 // cache would not fit in place).
-template <typename T>
-__global__ void __launch_bounds__(kRowThreads) ce_row_kernel(CeArgs a) {
+template <typename T, int NG>
+__global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
   constexpr int ES = Elem<T>::kBytes;
   constexpr int EPC = 16 / ES;
+  constexpr int NT = kRowThreads / NG;  // threads per group
+  constexpr int GW = NT / 32;           // warps per group
+  constexpr int L = NG == 1 ? 2 : 1;    // rows in flight per group (buffers)
   constexpr bool kBf16 = ES == 2;
   constexpr float kShift = kBf16 ? 14.0f : 0.0f;  // log2 of the fp16 cache scale
   extern __shared__ __align__(128) uint8_t smem[];
   RowShared& sh = *reinterpret_cast<RowShared*>(smem);
-  uint8_t* buf = smem + kHdrBytes;
-  const int tid = threadIdx.x;
-
+  const int grp = NG == 1 ? 0 : static_cast<int>(threadIdx.x) / NT;
+  const int tid = static_cast<int>(threadIdx.x) - grp * NT;  // thread within the group
+  const int lane = tid & 31, gwarp = tid >> 5;
+  const bool leader = tid == 0;
   const int S = a.cluster;
-  const int64_t row = blockIdx.x / S;
-  const int rank = static_cast<int>(blockIdx.x - row * S);
-  const int64_t V = a.V;
-  const int64_t e0 = static_cast<int64_t>(rank) * a.slice;
-  const int n = static_cast<int>(tmax<int64_t>(0, tmin<int64_t>(V, e0 + a.slice) - e0));
-  const int64_t t = a.targets[row];
-  const bool valid = (t != a.ignore_index) && t >= 0 && t < V;
-
-  const uint8_t* gsrc = reinterpret_cast<const uint8_t*>(a.logits) + (row * a.ld + e0) * ES;
-  uint8_t* gdst = reinterpret_cast<uint8_t*>(a.grad) + (row * a.ld + e0) * ES;
-
-  if (!valid) {
-    // Ignored row: zero gradient, zero loss, no read of the logits.  Every CTA
-    // of the cluster takes this branch, so no cluster barrier is entered.
-    if (rank == 0 && tid == 0) a.row_loss[row] = 0.0f;
-    const int glead = static_cast<int>(reinterpret_cast<uintptr_t>(gdst) & 15);
-    const int gspan = glead + n * ES;
-    const int c_lo = (glead + 15) >> 4, c_hi = max(c_lo, gspan >> 4);
-    uint8_t* gbase = gdst - glead;
-    for (int c = c_lo + tid; c < c_hi; c += kRowThreads)
-      *reinterpret_cast<uint4*>(gbase + 16 * c) = make_uint4(0, 0, 0, 0);
-    const int h = min(n, (16 * c_lo - glead) / ES);
-    const int kt = max(h, (16 * c_hi - glead) / ES);
-    for (int k = tid; k < h; k += kRowThreads) Elem<T>::store(gdst + k * ES, 0.0f);
-    for (int k = kt + tid; k < n; k += kRowThreads) Elem<T>::store(gdst + k * ES, 0.0f);
-    return;
-  }
-
-  // ---- issue the bulk loads ---------------------------------------------------------
-  // buf byte j <-> global byte (gsrc - lead + j); element k at buf[lead + k*ES].
-  const int lead = static_cast<int>(reinterpret_cast<uintptr_t>(gsrc) & 15);
-  const int span = lead + n * ES;
-  const int nchunks = (span + 15) >> 4;
-  const int c_lo = (lead + 15) >> 4;       // first chunk fully inside the slice
-  const int c_hi = max(c_lo, span >> 4);   // one past the last full chunk
-  const int nbulk = c_hi - c_lo;
-  const int npieces = nbulk == 0 ? 0 : max(1, min(kMaxPieces, nbulk / kMinPieceChunks));
-  const uint8_t* gbase = gsrc - lead;
-
-  if (tid == 0) {
-    for (int p = 0; p < npieces; ++p) mbar_init(&sh.bars[p], 1);
-    fence_mbar_init();
-    for (int p = 0; p < npieces; ++p) {
-      const int cs = c_lo + (nbulk * p) / npieces, ce = c_lo + (nbulk * (p + 1)) / npieces;
-      const uint32_t bytes = 16u * (ce - cs);
-      mbar_arrive_expect_tx(&sh.bars[p], bytes);
-      bulk_g2s(buf + 16 * cs, gbase + 16 * cs, bytes, &sh.bars[p]);
-    }
-  }
-  // The owners of the partial chunks at both ends fill them element by element
-  // and pad them with -inf (which contributes exp(-inf) = 0 everywhere).
-  auto fill_edge_chunk = [&](int c) {
-    for (int b = 16 * c; b < 16 * c + 16; b += ES) {
-      const int k = (b - lead) / ES;
-      T v = neg_inf_elem<T>();
-      if (b >= lead && k < n) v = *reinterpret_cast<const T*>(gsrc + k * ES);
-      *reinterpret_cast<T*>(buf + b) = v;
-    }
+  const int cid = blockIdx.x / S;
+  const int rank = blockIdx.x - cid * S;
+  const int64_t ngroups = static_cast<int64_t>(gridDim.x / S) * NG;
+  const int64_t first = static_cast<int64_t>(cid) * NG + grp;
+  auto gsync = [&]() {
+    if constexpr (NG == 1) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(NT) : "memory");
   };
-  for (int c = tid; c < c_lo; c += kRowThreads) fill_edge_chunk(c);
-  for (int c = c_hi + tid; c < nchunks; c += kRowThreads) fill_edge_chunk(c);
-  __syncthreads();  // barriers initialised before anyone waits on them
+  auto slot_of = [&](int64_t k) { return NG == 1 ? static_cast<int>(k & 1) : grp; };
+  auto buf_of = [&](int slot) { return smem + kHdrBytes + slot * a.buf_bytes; };
+  auto row_of = [&](int64_t k) { return first + k * ngroups; };
+  auto tgt_of = [&](int64_t k) { return row_of(k) < a.B ? a.targets[row_of(k)] : int64_t(0); };
 
-  // ---- pass 0: max ---------------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    for (int sl = 0; sl < 2; ++sl)
+      for (int p = 0; p < kPieces; ++p) mbar_init(&sh.full[sl][p], 1);
+    fence_mbar_init();
+  }
+  if (leader) {
+    sh.tgt[grp][0] = tgt_of(0);
+    sh.tgt[grp][1] = tgt_of(1);
+  }
+  __syncthreads();
+  if (leader)
+    for (int64_t k = 0; k < L; ++k) issue_slice<ES>(a, row_of(k), sh.tgt[grp][k & 1], rank, buf_of(slot_of(k)),
+                                                    sh.full[slot_of(k)]);
+
+  uint32_t phase = 0;       // bit sl: parity of the next waits on slot sl
+  uint32_t valid_rows = 0;  // selects the cluster record buffer
   bool ok = true;
-  float m_thr;
-  if constexpr (kBf16) {
-    uint32_t mx = 0xff80ff80u;  // packed (-inf, -inf)
-    auto fold_max = [&](int c) {
-      const uint4 q = *reinterpret_cast<const uint4*>(buf + 16 * c);
-      mx = bf16x2_max(mx, bf16x2_max(bf16x2_max(q.x, q.y), bf16x2_max(q.z, q.w)));
-    };
-    for (int c = tid; c < c_lo; c += kRowThreads) fold_max(c);
-    for (int c = c_hi + tid; c < nchunks; c += kRowThreads) fold_max(c);
-    for (int p = 0; p < npieces; ++p) {
-      const int cs = c_lo + (nbulk * p) / npieces, ce = c_lo + (nbulk * (p + 1)) / npieces;
-      if (!mbar_wait(&sh.bars[p], 0)) ok = false;
-      int c = cs + ((tid - cs) % kRowThreads + kRowThreads) % kRowThreads;
-      for (; c < ce; c += kRowThreads) fold_max(c);
-    }
-    m_thr = fmaxf(bf16_lo(mx), bf16_hi(mx));
-  } else {
-    m_thr = kNegInf;
-    auto fold_max = [&](int c) {
-      const float4 q = *reinterpret_cast<const float4*>(buf + 16 * c);
-      m_thr = fmaxf(m_thr, fmaxf(fmaxf(q.x, q.y), fmaxf(q.z, q.w)));
-    };
-    for (int c = tid; c < c_lo; c += kRowThreads) fold_max(c);
-    for (int c = c_hi + tid; c < nchunks; c += kRowThreads) fold_max(c);
-    for (int p = 0; p < npieces; ++p) {
-      const int cs = c_lo + (nbulk * p) / npieces, ce = c_lo + (nbulk * (p + 1)) / npieces;
-      if (!mbar_wait(&sh.bars[p], 0)) ok = false;
-      int c = cs + ((tid - cs) % kRowThreads + kRowThreads) % kRowThreads;
-      for (; c < ce; c += kRowThreads) fold_max(c);
-    }
-  }
-  const float m_cta = block_max<kRowThreads>(m_thr, sh.red_m);
-
-  // ---- pass 1: sum of exp(x - m); bf16 rows cache 2^14 * exp(x - m) as fp16 ------------
-  const int64_t tl = t - e0;  // target position within this slice
-  const bool has_t = tl >= 0 && tl < n;
-  const int tpos = has_t ? lead + static_cast<int>(tl) * ES : -1;  // byte position of the target
-  // m_cta = -inf only for an empty slice; every exponent is then exp(-inf) = 0.
-  const float nm = (m_cta == kNegInf) ? 0.0f : fmaf(-m_cta, kLog2e, kShift);
-  float s_thr = 0.0f;
-  for (int c = tid; c < nchunks; c += kRowThreads) {
-    uint4* p = reinterpret_cast<uint4*>(buf + 16 * c);
-    float v[EPC];
-    unpack16<T>(*p, v);
-    if ((tpos >> 4) == c) {
-      const int ti = (tpos & 15) / ES;
-#pragma unroll
-      for (int i = 0; i < EPC; ++i)
-        if (i == ti) sh.xt_local = v[i];
-    }
-    float e[EPC];
-#pragma unroll
-    for (int i = 0; i < EPC; ++i) e[i] = ex2(fmaf(v[i], kLog2e, nm));
-    s_thr += tree_sum(e);
-    if constexpr (kBf16) *p = pack_f16x8(e);
-  }
-  const float s_cta = block_sum<kRowThreads>(s_thr, sh.red_s) * (kBf16 ? (1.0f / 16384.0f) : 1.0f);
-
-  // ---- combine across the cluster -----------------------------------------------------------
-  float lse, xt;
-  if (S == 1) {
-    lse = m_cta + logf(s_cta);
-    xt = sh.xt_local;
-  } else {
-    if (tid == 0) {
-      sh.rec_m = m_cta;
-      sh.rec_s = s_cta;
-      sh.rec_has_t = has_t ? 1 : 0;
-      sh.rec_xt = has_t ? sh.xt_local : 0.0f;
-    }
-    cluster_arrive_release();
-    cluster_wait_acquire();
-    if (tid == 0) {
-      MaxSum tot{kNegInf, 0.0f};
-      float x = 0.0f;
-      for (int r = 0; r < S; ++r) {  // fixed rank order: identical on every CTA
-        MaxSum pr{ld_dsmem_f32(map_to_rank(&sh.rec_m, r)), ld_dsmem_f32(map_to_rank(&sh.rec_s, r))};
-        tot = combine(tot, pr);
-        if (ld_dsmem_s32(map_to_rank(&sh.rec_has_t, r))) x = ld_dsmem_f32(map_to_rank(&sh.rec_xt, r));
-      }
-      sh.lse = tot.m + logf(tot.s);
-      sh.xt = x;
-    }
-    cluster_arrive_release();  // this CTA is done reading its peers
-    __syncthreads();
-    lse = sh.lse;
-    xt = sh.xt;
-  }
-  if (rank == 0 && tid == 0) a.row_loss[row] = (lse - xt) + a.z * lse * lse;
-
-  // ---- pass 2: gradient straight to global ----------------------------------------------------
   const unsigned long long nv = *a.n_valid;
   const float scale = a.mean ? 1.0f / static_cast<float>(nv > 0 ? nv : 1ull) : 1.0f;
-  const float coef = scale * (1.0f + 2.0f * a.z * lse);
-  // bf16: g = coef * exp(x - lse) = k * (2^14 exp(x - m)), k = coef * 2^-14 * exp(m - lse)
-  // fp32: g = coef * 2^(x log2e - lse log2e)
-  const float k = (m_cta == kNegInf) ? 0.0f : coef * ex2(fmaf(m_cta - lse, kLog2e, -kShift));
-  const float nl = -lse * kLog2e;
-  uint8_t* dbase = gdst - lead;
-  if (ok) {
-    for (int c = tid; c < nchunks; c += kRowThreads) {
-      const uint4 q = *reinterpret_cast<const uint4*>(buf + 16 * c);
-      float g[EPC];
+
+  for (int64_t k = 0; row_of(k) < a.B; ++k) {
+    const int64_t row = row_of(k);
+    const int sl = slot_of(k);
+    uint8_t* buf = buf_of(sl);
+    const int64_t t = sh.tgt[grp][k & 1];
+    // the leader fetches the target of row k + 2 early; it is stored after this row
+    const int64_t t_ahead = leader ? tgt_of(k + 2) : 0;
+    const SliceGeo g = slice_geo<ES>(a, row, rank);
+
+    if (!target_valid(a, t)) {
+      // Ignored row: zero gradient, zero loss, the logits are never read.
+      if (rank == 0 && leader) a.row_loss[row] = 0.0f;
+      const int glead = static_cast<int>(reinterpret_cast<uintptr_t>(g.gdst) & 15);
+      const int gspan = glead + g.n * ES;
+      const int z_lo = (glead + 15) >> 4, z_hi = max(z_lo, gspan >> 4);
+      uint8_t* zb = g.gdst - glead;
+      for (int c = z_lo + tid; c < z_hi; c += NT) *reinterpret_cast<uint4*>(zb + 16 * c) = make_uint4(0, 0, 0, 0);
+      const int h = min(g.n, (16 * z_lo - glead) / ES);
+      const int kt = max(h, (16 * z_hi - glead) / ES);
+      for (int e = tid; e < h; e += NT) Elem<T>::store(g.gdst + e * ES, 0.0f);
+      for (int e = kt + tid; e < g.n; e += NT) Elem<T>::store(g.gdst + e * ES, 0.0f);
+    } else {
+      // ---- pass 0: this thread's max, piece by piece as copies land ----------------------
+      const int nb = g.x_hi - g.x_lo;
+      const int np = npieces_of(nb);
+      // ragged ends outside the bulk range: element loads by their owners
+      auto fill_edge = [&](int c) {
+        for (int bb = 16 * c; bb < 16 * c + 16; bb += ES) {
+          const int e = (bb - g.lead) / ES;
+          T v = neg_inf_elem<T>();
+          if (bb >= g.lead && e < g.n) v = *reinterpret_cast<const T*>(g.gsrc + e * ES);
+          *reinterpret_cast<T*>(buf + bb) = v;
+        }
+      };
+      uint32_t mx0 = 0xff80ff80u, mx1 = 0xff80ff80u;  // bf16: packed (-inf, -inf)
+      float mf = kNegInf;                              // fp32
+      auto fold_max = [&](int c) {
+        const uint4 q = *reinterpret_cast<const uint4*>(buf + 16 * c);
+        if constexpr (kBf16) {
+          mx0 = bf16x2_max(mx0, bf16x2_max(bf16x2_max(q.x, q.y), bf16x2_max(q.z, q.w)));
+        } else {
+          mf = fmaxf(mf, fmaxf(fmaxf(__uint_as_float(q.x), __uint_as_float(q.y)),
+                               fmaxf(__uint_as_float(q.z), __uint_as_float(q.w))));
+        }
+      };
+      for (int c = tid; c < g.x_lo; c += NT) {
+        fill_edge(c);
+        fold_max(c);
+      }
+      for (int c = g.x_hi + ((tid - g.x_hi) % NT + NT) % NT; c < g.nchunks; c += NT) {
+        fill_edge(c);
+        fold_max(c);
+      }
+      for (int p = 0; p < np; ++p) {
+        const int cs = g.x_lo + (nb * p) / np, ce = g.x_lo + (nb * (p + 1)) / np;
+        if (!mbar_wait(&sh.full[sl][p], (phase >> sl) & 1)) ok = false;
+        // bulk-copied ragged ends: overwrite the bytes outside the slice with -inf
+        if (p == 0 && g.x_lo == 0 && g.lead > 0 && tid == 0)
+          for (int bb = 0; bb < g.lead; bb += ES) *reinterpret_cast<T*>(buf + bb) = neg_inf_elem<T>();
+        if (p == np - 1 && g.x_hi == g.nchunks && (g.span & 15) && tid == (g.nchunks - 1) % NT)
+          for (int bb = g.span; bb < 16 * g.nchunks; bb += ES) *reinterpret_cast<T*>(buf + bb) = neg_inf_elem<T>();
+        int c = cs + ((tid - cs) % NT + NT) % NT;
+        for (; c + NT < ce; c += 2 * NT) {
+          fold_max(c);
+          if constexpr (kBf16) {
+            const uint4 q = *reinterpret_cast<const uint4*>(buf + 16 * (c + NT));
+            mx1 = bf16x2_max(mx1, bf16x2_max(bf16x2_max(q.x, q.y), bf16x2_max(q.z, q.w)));
+          } else {
+            fold_max(c + NT);
+          }
+        }
+        if (c < ce) fold_max(c);
+      }
+      if (np > 0) phase ^= 1u << sl;
+      float m_t;
       if constexpr (kBf16) {
-        unpack_f16x8(q, g);
-#pragma unroll
-        for (int i = 0; i < EPC; ++i) g[i] *= k;
+        mx0 = bf16x2_max(mx0, mx1);
+        m_t = fmaxf(bf16_lo(mx0), bf16_hi(mx0));
       } else {
-        float v[EPC];
-        unpack16<T>(q, v);
-#pragma unroll
-        for (int i = 0; i < EPC; ++i) g[i] = coef * ex2(fmaf(v[i], kLog2e, nl));
+        m_t = mf;
       }
-      if ((tpos >> 4) == c) {
-        const int ti = (tpos & 15) / ES;
+
+      // ---- target logit (its owner reads it before pass 1 overwrites the chunk) -----------
+      const int64_t tl = t - static_cast<int64_t>(rank) * a.slice;  // target position in this slice
+      const bool has_t = tl >= 0 && tl < g.n;
+      const int tpos = has_t ? g.lead + static_cast<int>(tl) * ES : -1;
+      const bool own_t = has_t && ((tpos >> 4) % NT) == tid;
+      if (own_t) sh.xt_local[grp] = Elem<T>::load(buf + tpos);
+
+      // ---- pass 1: sum of exp(x - m_t); bf16 rows cache 2^14 exp(x - m_t) as fp16 --------
+      const float nm = (m_t == kNegInf) ? 0.0f : fmaf(-m_t, kLog2e, kShift);
+      float s_t;
+      {
+        const float2 l2 = make_float2(kLog2e, kLog2e), nm2 = make_float2(nm, nm);
+        float2 acc = make_float2(0.0f, 0.0f);
+        auto exps = [&](const uint4& q, float (&e)[EPC]) {
+          float v[EPC];
+          unpack16<T>(q, v);
 #pragma unroll
-        for (int i = 0; i < EPC; ++i)
-          if (i == ti) g[i] -= scale;
+          for (int j = 0; j < EPC; j += 2) {
+            const float2 y = __ffma2_rn(make_float2(v[j], v[j + 1]), l2, nm2);
+            e[j] = ex2(y.x);
+            e[j + 1] = ex2(y.y);
+          }
+#pragma unroll
+          for (int j = 0; j < EPC; j += 2) acc = __fadd2_rn(acc, make_float2(e[j], e[j + 1]));
+        };
+        int c = tid;
+        for (; c + NT < g.nchunks; c += 2 * NT) {
+          uint4* p0 = reinterpret_cast<uint4*>(buf + 16 * c);
+          uint4* p1 = reinterpret_cast<uint4*>(buf + 16 * (c + NT));
+          const uint4 q0 = *p0, q1 = *p1;
+          float e0[EPC], e1[EPC];
+          exps(q0, e0);
+          exps(q1, e1);
+          if constexpr (kBf16) {
+            *p0 = pack_f16x8(e0);
+            *p1 = pack_f16x8(e1);
+          }
+        }
+        if (c < g.nchunks) {
+          uint4* p0 = reinterpret_cast<uint4*>(buf + 16 * c);
+          float e0[EPC];
+          exps(*p0, e0);
+          if constexpr (kBf16) *p0 = pack_f16x8(e0);
+        }
+        s_t = acc.x + acc.y;
       }
-      if (a.congruent && c >= c_lo && c < c_hi) {
-        *reinterpret_cast<uint4*>(dbase + 16 * c) = pack16<T>(g);
-      } else {
+
+      // ---- combine (m_t, s_t) over the group, then over the cluster ------------------------
+      MaxSum ms{m_t, s_t};
 #pragma unroll
-        for (int i = 0; i < EPC; ++i) {
-          const int kk = (16 * c + i * ES - lead) / ES;
-          if (16 * c + i * ES >= lead && kk < n) Elem<T>::store(gdst + kk * ES, g[i]);
+      for (int o = 16; o > 0; o >>= 1) {
+        MaxSum other{__shfl_xor_sync(0xffffffffu, ms.m, o), __shfl_xor_sync(0xffffffffu, ms.s, o)};
+        ms = combine(ms, other);
+      }
+      float* red_m = sh.red_m + grp * GW;
+      float* red_s = sh.red_s + grp * GW;
+      if (lane == 0) {
+        red_m[gwarp] = ms.m;
+        red_s[gwarp] = ms.s;
+      }
+      gsync();
+      const int rb = valid_rows & 1;
+      if (gwarp == 0) {
+        MaxSum w = lane < GW ? MaxSum{red_m[lane], red_s[lane]} : MaxSum{kNegInf, 0.0f};
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          MaxSum other{__shfl_xor_sync(0xffffffffu, w.m, o), __shfl_xor_sync(0xffffffffu, w.s, o)};
+          w = combine(w, other);
+        }
+        if (lane == 0) {
+          const float s_cta = w.s * (kBf16 ? (1.0f / 16384.0f) : 1.0f);
+          if (S == 1) {
+            sh.lse[grp] = w.m + logf(s_cta);
+            sh.xt[grp] = sh.xt_local[grp];
+          } else {
+            sh.rec_m[rb] = w.m;
+            sh.rec_s[rb] = s_cta;
+            sh.rec_has_t[rb] = has_t ? 1 : 0;
+            sh.rec_xt[rb] = has_t ? sh.xt_local[grp] : 0.0f;
+            fence_cluster();  // the record is visible cluster-wide before this thread arrives
+          }
+        }
+      }
+      if constexpr (NG == 1) {
+        if (S > 1) {
+          cluster_arrive_relaxed();
+          cluster_wait_acquire();
+          if (leader) {
+            MaxSum tot{kNegInf, 0.0f};
+            float x = 0.0f;
+            for (int r = 0; r < S; ++r) {  // fixed rank order: identical on every CTA
+              MaxSum pr{ld_dsmem_f32(map_to_rank(&sh.rec_m[rb], r)), ld_dsmem_f32(map_to_rank(&sh.rec_s[rb], r))};
+              tot = combine(tot, pr);
+              if (ld_dsmem_s32(map_to_rank(&sh.rec_has_t[rb], r))) x = ld_dsmem_f32(map_to_rank(&sh.rec_xt[rb], r));
+            }
+            sh.lse[0] = tot.m + logf(tot.s);
+            sh.xt[0] = x;
+          }
+        }
+      }
+      gsync();
+      const float lse = sh.lse[grp];
+      ++valid_rows;
+      if (rank == 0 && leader) a.row_loss[row] = (lse - sh.xt[grp]) + a.z * lse * lse;
+
+      // ---- pass 2: gradient straight to global -------------------------------------------
+      const float coef = scale * (1.0f + 2.0f * a.z * lse);
+      const float k_t = (m_t == kNegInf) ? 0.0f : coef * ex2(fmaf(m_t - lse, kLog2e, -kShift));
+      const float nl = -lse * kLog2e;
+      const float2 k2 = make_float2(k_t, k_t);
+      auto grad16 = [&](const uint4& q, float (&gv)[EPC]) {
+        if constexpr (kBf16) {
+          float e[EPC];
+          unpack_f16x8(q, e);
+#pragma unroll
+          for (int j = 0; j < EPC; j += 2) {
+            const float2 r = __fmul2_rn(make_float2(e[j], e[j + 1]), k2);
+            gv[j] = r.x;
+            gv[j + 1] = r.y;
+          }
+        } else {
+          float v[EPC];
+          unpack16<T>(q, v);
+#pragma unroll
+          for (int j = 0; j < EPC; ++j) gv[j] = coef * ex2(fmaf(v[j], kLog2e, nl));
+        }
+      };
+      auto store_elems = [&](int c, const float (&gv)[EPC]) {
+#pragma unroll
+        for (int j = 0; j < EPC; ++j) {
+          const int e = (16 * c + j * ES - g.lead) / ES;
+          if (16 * c + j * ES >= g.lead && e < g.n) Elem<T>::store(g.gdst + e * ES, gv[j]);
+        }
+      };
+      if (ok) {
+        if (a.congruent) {
+          uint8_t* dbase = g.gdst - g.lead;
+          int c = g.c_lo + ((tid - g.c_lo) % NT + NT) % NT;
+          for (; c + NT < g.c_hi; c += 2 * NT) {
+            const uint4 q0 = *reinterpret_cast<const uint4*>(buf + 16 * c);
+            const uint4 q1 = *reinterpret_cast<const uint4*>(buf + 16 * (c + NT));
+            float g0[EPC], g1[EPC];
+            grad16(q0, g0);
+            grad16(q1, g1);
+            *reinterpret_cast<uint4*>(dbase + 16 * c) = pack16<T>(g0);
+            *reinterpret_cast<uint4*>(dbase + 16 * (c + NT)) = pack16<T>(g1);
+          }
+          if (c < g.c_hi) {
+            const uint4 q0 = *reinterpret_cast<const uint4*>(buf + 16 * c);
+            float g0[EPC];
+            grad16(q0, g0);
+            *reinterpret_cast<uint4*>(dbase + 16 * c) = pack16<T>(g0);
+          }
+          for (int ce = tid; ce < g.c_lo; ce += NT) {
+            float g0[EPC];
+            grad16(*reinterpret_cast<const uint4*>(buf + 16 * ce), g0);
+            store_elems(ce, g0);
+          }
+          for (int ce = g.c_hi + ((tid - g.c_hi) % NT + NT) % NT; ce < g.nchunks; ce += NT) {
+            float g0[EPC];
+            grad16(*reinterpret_cast<const uint4*>(buf + 16 * ce), g0);
+            store_elems(ce, g0);
+          }
+        } else {
+          for (int c = tid; c < g.nchunks; c += NT) {
+            float g0[EPC];
+            grad16(*reinterpret_cast<const uint4*>(buf + 16 * c), g0);
+            store_elems(c, g0);
+          }
+        }
+        if (own_t) {  // the target element, rewritten after its chunk with the -scale term
+          float gt;
+          if constexpr (kBf16) {
+            gt = k_t * f16_to_f32(*reinterpret_cast<const uint16_t*>(buf + tpos));
+          } else {
+            gt = coef * ex2(fmaf(sh.xt_local[grp], kLog2e, nl));
+          }
+          Elem<T>::store(g.gdst + tl * ES, gt - scale);
         }
       }
     }
+    // The buffer is free once every thread of the group is past this row; its
+    // generic-proxy writes are ordered before the bulk copy that refills it.
+    fence_proxy_async_smem();
+    gsync();
+    if (leader) {
+      sh.tgt[grp][k & 1] = t_ahead;  // row k + 2's target (row k + 1's is already stored)
+      const int64_t kn = k + L;      // next row into this slot
+      issue_slice<ES>(a, row_of(kn), L == 2 ? t_ahead : sh.tgt[grp][kn & 1], rank, buf, sh.full[sl]);
+    }
   }
-  if (S > 1) cluster_wait_acquire();  // peers have finished reading this CTA's record
+  if constexpr (NG == 1) {
+    if (S > 1) {  // no CTA leaves while a peer may still read its records
+      cluster_arrive_relaxed();
+      cluster_wait_acquire();
+    }
+  }
 }
 
 // Rows too long for the shared-memory path: one CTA per row, two passes over
@@ -580,50 +801,142 @@ __global__ void __launch_bounds__(1024) ce_reduce_kernel(const float* __restrict
 // host side
 // ------------------------------------------------------------------------------
 
-static int ce_max_slice_bytes() {
-  // Slices up to 64 KiB keep three or more row-CTAs resident per SM.
+static int ce_slice_target_bytes() {
+  // Largest slice before a row is split across a cluster (tunable for sweeps).
   static int v = [] {
     const char* e = std::getenv("GH_CE_SLICE_KB");
-    int kb = e ? std::atoi(e) : 64;
-    return std::min(std::max(kb, 4), 200) * 1024;
+    const int kb = e ? std::atoi(e) : 110;
+    return std::min(std::max(kb, 4), kMaxSliceBytes / 1024) * 1024;
   }();
   return v;
 }
 
 CePlan ce_plan(int64_t V, int elem_bytes) {
   CePlan p{};
-  const int64_t max_slice = ce_max_slice_bytes();
-  int S = 1;
+  const int64_t target = ce_slice_target_bytes();
   auto slice_for = [&](int s) {
-    int64_t q = (V + s - 1) / s;
+    const int64_t q = (V + s - 1) / s;
     return ((q + 15) / 16) * 16;  // slices start on 32/64-byte boundaries of the row
   };
-  while (S < 8 && slice_for(S) * elem_bytes > max_slice) S *= 2;
-  int64_t q = slice_for(S);
-  if (q * elem_bytes > 200 * 1024) {
+  int S = 1;
+  while (S < 8 && slice_for(S) * elem_bytes > target) S *= 2;
+  const int64_t q = slice_for(S);
+  if (q * elem_bytes > kMaxSliceBytes) {
     p.streaming = true;
     p.cluster = 1;
-    p.slice = 0;
-    p.smem_bytes = 0;
     return p;
   }
   p.streaming = false;
   p.cluster = S;
   p.slice = static_cast<int>(q);
   const int64_t chunks = (15 + q * elem_bytes + 15) / 16 + 1;
-  p.smem_bytes = static_cast<int>(kHdrBytes + 16 * chunks);
+  p.buf_bytes = static_cast<int>(((16 * chunks) + 127) / 128 * 128);
+  p.smem_bytes = kHdrBytes + 2 * p.buf_bytes;
   return p;
 }
 
+static int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+namespace {
+
+// Rows of one slice run two row groups per CTA; rows split over a cluster run
+// one double-buffered group.
+void (*row_kernel_for(int es, int cluster))(CeArgs) {
+  if (es == 4) return cluster == 1 ? ce_row_kernel<float, 2> : ce_row_kernel<float, 1>;
+  return cluster == 1 ? ce_row_kernel<uint16_t, 2> : ce_row_kernel<uint16_t, 1>;
+}
+
+// Launch plan of the row kernel for one (device, V, element size), computed
+// once: the occupancy queries and attribute calls cost far more than a launch.
+struct PlanEntry {
+  int dev;
+  int64_t V;
+  int es;
+  CePlan plan;
+  int64_t active;  // resident clusters
+};
+
+std::mutex g_plan_mu;
+PlanEntry g_plans[64];
+int g_nplans = 0;
+
+gh_status_t row_plan(int64_t V, int es, CePlan* out, int64_t* active_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GH_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_plan_mu);
+  for (int i = 0; i < g_nplans; ++i) {
+    if (g_plans[i].dev == dev && g_plans[i].V == V && g_plans[i].es == es) {
+      *out = g_plans[i].plan;
+      *active_out = g_plans[i].active;
+      return GH_OK;
+    }
+  }
+  const CePlan plan = ce_plan(V, es);
+  int64_t active = 0;
+  if (!plan.streaming) {
+    void (*kern)(CeArgs) = row_kernel_for(es, plan.cluster);
+    // The dynamic shared memory limit is an attribute of the kernel, shared by
+    // every plan: raise it once per device to the opt-in maximum.
+    static bool raised[64][2][2] = {};
+    const int kv = es == 4, kg = plan.cluster == 1;
+    if (dev < 64 && !raised[dev][kv][kg]) {
+      int optin = 0;
+      if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return GH_ERR_CUDA;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
+        return GH_ERR_CUDA;
+      raised[dev][kv][kg] = true;
+    }
+    if (plan.smem_bytes > kHdrBytes + 2 * (kMaxSliceBytes + 256)) return GH_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kRowThreads);
+    cfg.dynamicSmemBytes = plan.smem_bytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = plan.cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.cluster * device_sm_count()));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    active = n;
+    if (active <= 0) return GH_ERR_UNSUPPORTED;
+  }
+  if (std::getenv("GH_DEBUG_PLAN"))
+    std::fprintf(stderr, "gh ce plan: V=%lld es=%d streaming=%d cluster=%d slice=%d buf=%d smem=%d clusters=%lld\n",
+                 static_cast<long long>(V), es, plan.streaming ? 1 : 0, plan.cluster, plan.slice, plan.buf_bytes,
+                 plan.smem_bytes, static_cast<long long>(active));
+  if (g_nplans < 64) g_plans[g_nplans++] = PlanEntry{dev, V, es, plan, active};
+  *out = plan;
+  *active_out = active;
+  return GH_OK;
+}
+
+}  // namespace
+
 gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaStream_t stream) {
   CeArgs a = args_in;
+  a.B = B;
   const int es = dtype == GH_F32 ? 4 : 2;
-  const CePlan plan = ce_plan(a.V, es);
+  CePlan plan;
+  int64_t active = 0;
+  gh_status_t st = row_plan(a.V, es, &plan, &active);
+  if (st != GH_OK) return st;
   a.cluster = plan.cluster;
   a.slice = plan.slice;
+  a.buf_bytes = plan.buf_bytes;
 
-  if (B * plan.cluster > INT32_MAX) return GH_ERR_UNSUPPORTED;  // one grid covers every row
   if (plan.streaming) {
+    if (B > INT32_MAX) return GH_ERR_UNSUPPORTED;
     ProfileScope prof(GH_KERNEL_CE_ROW, stream);
     if (dtype == GH_F32) ce_stream_kernel<float><<<static_cast<unsigned>(B), kStreamThreads, 0, stream>>>(a);
     else ce_stream_kernel<uint16_t><<<static_cast<unsigned>(B), kStreamThreads, 0, stream>>>(a);
@@ -631,11 +944,8 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
     return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
   }
 
-  void (*kern)(CeArgs) = dtype == GH_F32 ? ce_row_kernel<float> : ce_row_kernel<uint16_t>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem_bytes) != cudaSuccess)
-    return GH_ERR_CUDA;
+  void (*kern)(CeArgs) = row_kernel_for(es, plan.cluster);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(B * plan.cluster));
   cfg.blockDim = dim3(kRowThreads);
   cfg.dynamicSmemBytes = plan.smem_bytes;
   cfg.stream = stream;
@@ -646,6 +956,11 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // Persistent grid: as many clusters as can be resident at once, no more
+  // than there are rows (two per CTA with two row groups).
+  const int64_t per_cluster = plan.cluster == 1 ? 2 : 1;
+  const int64_t nclusters = std::min<int64_t>(active, (B + per_cluster - 1) / per_cluster);
+  cfg.gridDim = dim3(static_cast<unsigned>(nclusters * plan.cluster));
   ProfileScope prof(GH_KERNEL_CE_ROW, stream);
   note_launch();
   if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return GH_ERR_CUDA;
@@ -654,8 +969,13 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
 
 gh_status_t ce_count_launch(const int64_t* targets, int64_t n, int64_t V, int64_t ii,
                             unsigned long long* count, cudaStream_t stream) {
+  if (n <= (int64_t(1) << 20)) {
+    // one CTA counts without atomics and writes the counter itself
+    ce_count1_kernel<<<1, 1024, 0, stream>>>(targets, n, V, ii, count);
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+  }
   if (cudaMemsetAsync(count, 0, sizeof(unsigned long long), stream) != cudaSuccess) return GH_ERR_CUDA;
-  if (n == 0) return GH_OK;
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 4);
   ce_count_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(targets, n, V, ii, count);
   note_launch();

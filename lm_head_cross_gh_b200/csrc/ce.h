@@ -19,8 +19,10 @@ struct CeArgs {
   int mean;                           // 1: divide by n_valid
   const unsigned long long* n_valid;  // written by ce_count_kernel
   float* row_loss;                    // [B] scratch
+  int64_t B;                          // rows (set by ce_launch)
   int slice;                          // elements per CTA (set by ce_launch)
   int cluster;                        // CTAs per row (set by ce_launch)
+  int buf_bytes;                      // bytes per slice buffer (set by ce_launch)
   int congruent;                      // (logits - grad) % 16 == 0
 };
 
@@ -28,6 +30,7 @@ struct CePlan {
   bool streaming;  // row too long for the shared-memory path
   int cluster;     // CTAs per row
   int slice;       // elements per CTA
+  int buf_bytes;   // one slice buffer (two per CTA)
   int smem_bytes;  // dynamic shared memory per CTA
 };
 

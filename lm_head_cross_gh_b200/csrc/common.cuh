@@ -19,9 +19,15 @@ __device__ __forceinline__ void record_status(int code) {
   atomicCAS(&g_device_status, 0, code);
 }
 
-// Iteration bound of every device-side spin: far above any legitimate wait
-// (each try_wait blocks for a hardware-defined slice) yet finite.
-constexpr uint32_t kSpinLimit = 1u << 24;
+// Every device-side wait gives up after kWaitTimeoutNs of wall time (read
+// from %globaltimer): far above any legitimate wait, yet finite.
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -46,24 +52,29 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
+// One potentially blocking test of phase `parity`: the thread may be
+// suspended in hardware (not spinning) for up to `suspend_ns` while it waits.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity, uint32_t suspend_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar_addr), "r"(parity)
+      : "r"(bar_addr), "r"(parity), "r"(suspend_ns)
       : "memory");
   return ok != 0;
 }
 
 // Bounded wait for phase `parity` of `bar` to complete.  Returns false (and
-// records GH_ERR_TIMEOUT) if the bound runs out.
+// records GH_ERR_TIMEOUT) once kWaitTimeoutNs has passed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(a, parity)) return true;
+  if (mbar_try_wait(a, parity, 100000u)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(a, parity, 100000u)) return true;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) break;
   }
   record_status(GH_ERR_TIMEOUT);
   return false;
@@ -113,9 +124,17 @@ __device__ __forceinline__ void cluster_arrive_release() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
 
+// Arrive without ordering this thread's earlier memory operations; pair with
+// fence_cluster() in the one thread whose writes the peers must see.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+
+__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 
 // Address of the same shared variable in CTA `rank` of this cluster.
 __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {

@@ -57,6 +57,16 @@ def test_cluster_paths(cuda_device, dtype, V, B):
     check_problem_full(p, loss, grad_to_f64(grad), f"cluster {dtype} V={V}")
 
 
+@pytest.mark.parametrize("dtype,V,B", [("bf16", 5003, 1500), ("f32", 30011, 700), ("bf16", 100003, 700),
+                                       ("bf16", 262147, 300)])
+def test_many_rows_per_persistent_cta(cuda_device, dtype, V, B):
+    # more rows than resident CTAs: each CTA cycles both slice buffers many
+    # times, with ignored rows (no copy, no cluster exchange) interleaved
+    p = gh_synth.ce_normal(B, V, 3.0, dtype=dtype, ignore_frac=0.3, reduction="mean", z_loss=1e-4, seed=V)
+    loss, grad = run(p)
+    check_problem_full(p, loss, grad_to_f64(grad), f"persistent {dtype} V={V} B={B}")
+
+
 @pytest.mark.parametrize("dtype,V", [("bf16", 1_200_003), ("f32", 600_001)])
 def test_streaming_path_for_very_long_rows(cuda_device, dtype, V):
     p = gh_synth.ce_normal(3, V, 3.0, dtype=dtype, ignore_frac=0.0, reduction="sum", z_loss=1e-4, seed=4)
