@@ -101,6 +101,31 @@ gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B,
                           float z_mult, float* loss, void* grad, void* stream);
 
 /*
+ * gh_ce_fwd_bwd_noalloc — gh_ce_fwd_bwd for callers that cannot allocate.
+ * The pages have no counterpart; this entry point exists for callers whose
+ * device memory is already owned in full by another allocator (a framework's
+ * caching allocator, or a fixed arena planned ahead of time), where the
+ * cudaMallocAsync that gh_ce_fwd_bwd makes for its scratch could fail in the
+ * middle of a step, and for loops that forbid allocator calls inside a step.
+ *
+ * Arguments, results and errors are those of gh_ce_fwd_bwd, except:
+ *  - B is limited to 65536 rows: the scratch is a fixed array of
+ *    256 + 4 * 65536 bytes inside the library's device image, which every GPU
+ *    that loads the library keeps until the process exits.  Larger B returns
+ *    GH_ERR_UNSUPPORTED and enqueues nothing.
+ *  - The call makes no cudaMalloc/cudaFree and no allocating library call.
+ *  - The first call with a given device current looks up the array's device
+ *    address (cudaGetSymbolAddress) and caches it; make that first call
+ *    before any stream capture on that device.
+ *  - All calls share the one array and it keeps the last call's contents (the
+ *    call clears what must start at zero).  Calls whose GPU work overlaps
+ *    (different streams or host threads) race on it; serialise them.
+ */
+gh_status_t gh_ce_fwd_bwd_noalloc(const void* logits, const int64_t* targets, int64_t B, int64_t V,
+                                  gh_dtype_t dtype, int64_t ignore_index, gh_reduction_t reduction,
+                                  float z_mult, float* loss, void* grad, void* stream);
+
+/*
  * gh_linear_ce — chunked fused linear cross-entropy (Greyhound
  * `chunked_linear_cross_entropy` over `chunked_linear_loss`).
  *

@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
     L.gh_ce_fwd_bwd.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_int, c_float,
                                 c_void_p, c_void_p, c_void_p]
     L.gh_ce_fwd_bwd.restype = c_int
+    L.gh_ce_fwd_bwd_noalloc.argtypes = list(L.gh_ce_fwd_bwd.argtypes)
+    L.gh_ce_fwd_bwd_noalloc.restype = c_int
     L.gh_linear_ce.argtypes = [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int,
                                c_int64, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p]
     L.gh_linear_ce.restype = c_int
@@ -152,6 +154,36 @@ def gh_ce_fwd_bwd(logits, targets, ignore_index: int = -100, reduction: str = "m
     return loss, grad
 
 
+GH_NOALLOC_MAX_ROWS = 65536
+
+
+def gh_ce_fwd_bwd_noalloc(logits, targets, ignore_index: int = -100, reduction: str = "mean",
+                          z_loss: float = 0.0, *, grad, loss, stream=None):
+    """``gh_ce_fwd_bwd`` without any device allocation inside the library.
+
+    For callers that cannot allocate during a step (their device memory is
+    owned by another allocator, or allocator calls are forbidden there).  The
+    caller passes every output (``grad`` and the float32 scalar ``loss``);
+    the library's scratch is a fixed device array shared by all calls, so
+    calls that overlap on the GPU race.  ``B`` <= 65536.
+    """
+    import torch
+    _need(logits.dim() == 2 and logits.is_cuda and logits.is_contiguous(), "logits: contiguous CUDA [B, V]")
+    _need(logits.dtype in (torch.float32, torch.bfloat16), "logits dtype must be float32 or bfloat16")
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
+          and targets.shape == (logits.shape[0],), "targets: contiguous CUDA int64 [B]")
+    _need(reduction in GH_REDUCTION, "reduction must be 'mean' or 'sum'")
+    _need(grad.shape == logits.shape and grad.dtype == logits.dtype and grad.is_contiguous(), "grad mismatch")
+    _need(loss.dtype == torch.float32 and loss.numel() == 1 and loss.is_cuda, "loss must be a CUDA float32 scalar")
+    B, V = logits.shape
+    dtype = GH_F32 if logits.dtype == torch.float32 else GH_BF16
+    st = lib().gh_ce_fwd_bwd_noalloc(_ptr(logits), _ptr(targets), B, V, dtype, int(ignore_index),
+                                     GH_REDUCTION[reduction], float(z_loss), _ptr(loss), _ptr(grad),
+                                     _stream_handle(stream))
+    _check(st, "gh_ce_fwd_bwd_noalloc")
+    return loss, grad
+
+
 def gh_linear_ce(inputs, weight, targets, ignore_index: int = -100, reduction: str = "mean",
                  z_loss: float = 0.0, chunk: int = 0, accum: str = "fp32", *, grad_inputs=None,
                  grad_weight=None, loss=None, stream=None):
@@ -211,7 +243,7 @@ def gh_get_device_status(stream=None) -> int:
 
 __all__ = [
     "GhError", "lib", "header_symbols", "status_string", "gh_status_string", "gh_version",
-    "gh_ce_fwd_bwd", "gh_linear_ce", "gh_get_device_status", "gh_profile_enable", "gh_profile_read",
+    "gh_ce_fwd_bwd", "gh_ce_fwd_bwd_noalloc", "GH_NOALLOC_MAX_ROWS", "gh_linear_ce", "gh_get_device_status", "gh_profile_enable", "gh_profile_read",
     "gh_launch_count", "GH_KERNEL",
     "GH_OK", "GH_ERR_INVALID_ARG", "GH_ERR_UNSUPPORTED", "GH_ERR_ALLOC", "GH_ERR_CUDA",
     "GH_ERR_TIMEOUT", "GH_ERR_TARGET_RANGE", "GH_REDUCTION", "GH_ACCUM", "GH_F32", "GH_BF16",

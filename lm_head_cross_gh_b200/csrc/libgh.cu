@@ -3,3 +3,4 @@
 #include "ce.cu"
 #include "linear_ce.cu"
 #include "api.cu"
+#include "noalloc.cu"
