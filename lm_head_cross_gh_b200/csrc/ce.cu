@@ -937,7 +937,7 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
 
   if (plan.streaming) {
     if (B > INT32_MAX) return GH_ERR_UNSUPPORTED;
-    ProfileScope prof(GH_KERNEL_CE_ROW, stream);
+    ProfileScope prof(a.profile_kind, stream);
     if (dtype == GH_F32) ce_stream_kernel<float><<<static_cast<unsigned>(B), kStreamThreads, 0, stream>>>(a);
     else ce_stream_kernel<uint16_t><<<static_cast<unsigned>(B), kStreamThreads, 0, stream>>>(a);
     note_launch();
@@ -961,7 +961,7 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
   const int64_t per_cluster = plan.cluster == 1 ? 2 : 1;
   const int64_t nclusters = std::min<int64_t>(active, (B + per_cluster - 1) / per_cluster);
   cfg.gridDim = dim3(static_cast<unsigned>(nclusters * plan.cluster));
-  ProfileScope prof(GH_KERNEL_CE_ROW, stream);
+  ProfileScope prof(a.profile_kind, stream);
   note_launch();
   if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return GH_ERR_CUDA;
   return GH_OK;

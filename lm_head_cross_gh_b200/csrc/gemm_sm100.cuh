@@ -1,0 +1,375 @@
+// Persistent bf16 GEMM on the sm_100a tensor cores (tcgen05.mma, TMEM
+// accumulators, TMA operand loads), written for the three contractions of the
+// chunked linear cross-entropy (Greyhound `chunked_linear_loss`):
+//
+//   logits_c = X_c  W^T   A = X_c [rows, D]   K-major    B = W   [V, D]    K-major
+//   dX_c     = G_c  W     A = G_c [rows, V]   K-major    B = W   [V, D]    N-major
+//   dW      += G_c^T X_c  A = G_c^T           M-major    B = X_c [rows, D] N-major
+//
+// D[M, N] = sum_k A[m, k] B[n, k].  Tiles of 128 x kBN are computed by one CTA
+// (cta_group::1) in 64-wide K steps.  Warp roles:
+//   warp 0      TMA producer (one elected lane): A and B tiles into a ring of
+//               kStages shared-memory stages, 128-byte swizzled
+//   warp 1      TMEM allocator and MMA issuer (one lane): 4 x tcgen05.mma
+//               (M=128, N=kBN, K=16) per stage, commits release stages and
+//               publish finished accumulators
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
+//               the 32 TMEM lanes its warp id selects), conversion, stores
+// Two accumulators of kBN fp32 columns (all 512 TMEM columns) let the
+// epilogue of one tile overlap the MMAs of the next.  Every wait is bounded
+// (GH_ERR_TIMEOUT, then all roles stop and TMEM is freed).
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace gh {
+namespace sm100 {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;                       // one 128-byte swizzle row of bf16
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;        // 16 KiB
+constexpr int kBBytes = kBN * kBK * 2;        // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kGemmThreads = 192;
+constexpr int kTmemCols = 2 * kBN;            // two accumulators
+constexpr int kGemmSmem = 1024 /*align*/ + kStages * kStageBytes + 256 /*barriers*/;
+
+// Epilogue modes (what happens to the fp32 tile acc[128, kBN]).
+enum GemmEpi : int {
+  kEpiStoreBf16 = 0,  // out = bf16(tile)
+  kEpiAccWrite = 1,   // acc = tile                      (fp32 accumulator, first chunk)
+  kEpiAccAdd = 2,     // acc += tile
+  kEpiAccFinal = 3,   // out = bf16(acc + tile)          (last chunk)
+  kEpiBf16Add = 4     // out = bf16(float(out) + tile)   (accumulate in the bf16 output)
+};
+
+struct GemmArgs {
+  int M, N, K;
+  int tiles_m, tiles_n, num_kb;
+  int m_fastest;        // tile order: consecutive tiles share the B tile (1) or the A tile (0)
+  int epi;
+  void* out;            // bf16 [M, ld_out]
+  int64_t ld_out;
+  float* acc;           // fp32 [M, ld_acc]
+  int64_t ld_acc;
+  int m_limit, n_limit; // rows / columns actually stored (n_limit a multiple of 8)
+};
+
+// ---- PTX wrappers ----------------------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D(tmem) (+)= A(smem desc) x B(smem desc), bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading and
+// stride byte offsets (all >> 4), version 1, base offset 0, 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, M x N, majors.
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)            // D format: f32
+         | (1u << 7)          // A format: bf16
+         | (1u << 10)         // B format: bf16
+         | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Wait with an abort flag shared by all roles: returns false once any role
+// timed out (and records GH_ERR_TIMEOUT when this wait is the one that did).
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity, 20000u)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(a, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1;
+      record_status(GH_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// ---- the kernel --------------------------------------------------------------------
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                     GemmArgs g) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tmem_full = empty + kStages;
+  uint64_t* tmem_empty = tmem_full + 2;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_tiles = g.tiles_m * g.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tma_a);
+    prefetch_tmap(&tma_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_slot;
+
+  auto tile_coords = [&](int tile, int& mb, int& nb) {
+    if (g.m_fastest) {
+      mb = tile % g.tiles_m;
+      nb = tile / g.tiles_m;
+    } else {
+      nb = tile % g.tiles_n;
+      mb = tile / g.tiles_n;
+    }
+  };
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool run = true;
+      for (int tile = blockIdx.x; tile < num_tiles && run; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, mb, nb);
+        const int m0 = mb * kBM, n0 = nb * kBN;
+        for (int kb = 0; kb < g.num_kb; ++kb) {
+          if (!wait_or_abort(&empty[stage], phase ^ 1, abort_flag)) {
+            run = false;
+            break;
+          }
+          uint8_t* sa = stage_base + stage * kStageBytes;
+          uint8_t* sb = sa + kABytes;
+          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          const int k0 = kb * kBK;
+          if constexpr (A_MN) {
+            tma_load_2d(sa, &tma_a, &full[stage], m0, k0);
+            tma_load_2d(sa + 8192, &tma_a, &full[stage], m0 + 64, k0);
+          } else {
+            tma_load_2d(sa, &tma_a, &full[stage], k0, m0);
+          }
+          if constexpr (B_MN) {
+#pragma unroll
+            for (int j = 0; j < kBN / 64; ++j) tma_load_2d(sb + j * 8192, &tma_b, &full[stage], n0 + 64 * j, k0);
+          } else {
+            tma_load_2d(sb, &tma_b, &full[stage], k0, n0);
+          }
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc(kBM, kBN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool run = true;
+      for (int tile = blockIdx.x; tile < num_tiles && run; tile += gridDim.x) {
+        if (!wait_or_abort(&tmem_empty[acc], acc_phase ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kBN;
+        for (int kb = 0; kb < g.num_kb; ++kb) {
+          if (!wait_or_abort(&full[stage], phase, abort_flag)) {
+            run = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * kStageBytes);
+          const uint32_t sb = sa + kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            // K-major: the 16-wide K step moves 32 bytes along the swizzled row;
+            // M/N-major: it moves 16 rows (2 x 1024-byte swizzle atoms).
+            const uint64_t ad = A_MN ? smem_desc(sa + k * 2048, 8192, 1024) : smem_desc(sa + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          umma_commit(&empty[stage]);  // stage free once these MMAs have read it
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!run) break;
+        umma_commit(&tmem_full[acc]);  // accumulator complete
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r_local = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      int mb, nb;
+      tile_coords(tile, mb, nb);
+      if (!wait_or_abort(&tmem_full[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const int row = mb * kBM + r_local;
+      const bool row_ok = row < g.m_limit;
+      const uint32_t t_row = tmem_base + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int cc = 0; cc < kBN; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(t_row + cc, v);
+        tmem_ld_wait();
+        const int col0 = nb * kBN + cc;
+        if (!row_ok || col0 >= g.n_limit) continue;
+        const int ncols = min(32, g.n_limit - col0);  // a multiple of 8
+        if (g.epi == kEpiStoreBf16 || g.epi == kEpiBf16Add) {
+          uint16_t* o = reinterpret_cast<uint16_t*>(g.out) + static_cast<int64_t>(row) * g.ld_out + col0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j * 8 >= ncols) break;
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[j * 8 + e]);
+            if (g.epi == kEpiBf16Add) {
+              const uint4 prev = *reinterpret_cast<const uint4*>(o + j * 8);
+              f[0] += bf16_lo(prev.x); f[1] += bf16_hi(prev.x);
+              f[2] += bf16_lo(prev.y); f[3] += bf16_hi(prev.y);
+              f[4] += bf16_lo(prev.z); f[5] += bf16_hi(prev.z);
+              f[6] += bf16_lo(prev.w); f[7] += bf16_hi(prev.w);
+            }
+            *reinterpret_cast<uint4*>(o + j * 8) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                              pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+          }
+        } else {
+          float* a = g.acc + static_cast<int64_t>(row) * g.ld_acc + col0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j * 8 >= ncols) break;
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[j * 8 + e]);
+            if (g.epi != kEpiAccWrite) {
+              const float4 p0 = *reinterpret_cast<const float4*>(a + j * 8);
+              const float4 p1 = *reinterpret_cast<const float4*>(a + j * 8 + 4);
+              f[0] += p0.x; f[1] += p0.y; f[2] += p0.z; f[3] += p0.w;
+              f[4] += p1.x; f[5] += p1.y; f[6] += p1.z; f[7] += p1.w;
+            }
+            if (g.epi == kEpiAccFinal) {
+              uint16_t* o = reinterpret_cast<uint16_t*>(g.out) + static_cast<int64_t>(row) * g.ld_out + col0;
+              *reinterpret_cast<uint4*>(o + j * 8) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+            } else {
+              *reinterpret_cast<float4*>(a + j * 8) = make_float4(f[0], f[1], f[2], f[3]);
+              *reinterpret_cast<float4*>(a + j * 8 + 4) = make_float4(f[4], f[5], f[6], f[7]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tmem_empty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  // ---------------- teardown ----------------
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace sm100
+}  // namespace gh
