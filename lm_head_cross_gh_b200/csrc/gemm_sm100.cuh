@@ -37,27 +37,31 @@ constexpr int kBBytes = kBN * kBK * 2;        // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 2 * kBN;            // two accumulators
-constexpr int kGemmSmem = 1024 /*align*/ + kStages * kStageBytes + 256 /*barriers*/;
+constexpr int kStageOutBytes = 4096;          // one epilogue staging buffer: 32 rows x 128 bytes
+constexpr int kOutBytes = 4 * 2 * kStageOutBytes;  // 4 epilogue warps x 2 buffers
+constexpr int kGemmSmem = 1024 /*align*/ + kStages * kStageBytes + kOutBytes + 256 /*barriers*/;
 
-// Epilogue modes (what happens to the fp32 tile acc[128, kBN]).
+// Epilogue modes (what happens to the fp32 tile).  The first three go out
+// through the `tma_out` tensor map from a swizzled shared-memory staging
+// buffer per epilogue warp; TMA clips rows and columns outside the map.
 enum GemmEpi : int {
-  kEpiStoreBf16 = 0,  // out = bf16(tile)
-  kEpiAccWrite = 1,   // acc = tile                      (fp32 accumulator, first chunk)
-  kEpiAccAdd = 2,     // acc += tile
-  kEpiAccFinal = 3,   // out = bf16(acc + tile)          (last chunk)
-  kEpiBf16Add = 4     // out = bf16(float(out) + tile)   (accumulate in the bf16 output)
+  kEpiStoreBf16 = 0,  // out(bf16) = tile                       TMA store
+  kEpiStoreF32 = 1,   // out(f32)  = tile                       TMA store
+  kEpiAddF32 = 2,     // out(f32) += tile                       TMA reduce-add (in L2)
+  kEpiBf16Add = 3     // out = bf16(float(out) + tile), direct loads and stores (bf16 accumulator)
 };
 
 struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, num_kb;
+  int k_splits;         // K is cut into k_splits ranges of kb_per_split K-steps
+  int kb_per_split;
+  int split_rows;       // row offset in the output map between K splits
   int m_fastest;        // tile order: consecutive tiles share the B tile (1) or the A tile (0)
   int epi;
-  void* out;            // bf16 [M, ld_out]
+  void* out;            // kEpiBf16Add only: bf16 [M, ld_out]
   int64_t ld_out;
-  float* acc;           // fp32 [M, ld_acc]
-  int64_t ld_acc;
-  int m_limit, n_limit; // rows / columns actually stored (n_limit a multiple of 8)
+  int m_limit, n_limit; // kEpiBf16Add only: rows / columns stored (n_limit a multiple of 8)
 };
 
 // ---- PTX wrappers ----------------------------------------------------------------
@@ -69,6 +73,23 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* smem_src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+
+// Allow at most one committed bulk group still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
@@ -159,11 +180,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                     GemmArgs g) {
+                     const __grid_constant__ CUtensorMap tma_out, GemmArgs g) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* out_stage = smem + kStages * kStageBytes;  // 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(out_stage + kOutBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tmem_full = empty + kStages;
   uint64_t* tmem_empty = tmem_full + 2;
@@ -171,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_tiles = g.tiles_m * g.tiles_n;
+  const int num_tiles = g.tiles_m * g.tiles_n * g.k_splits;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -186,6 +208,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&tma_a);
     prefetch_tmap(&tma_b);
+    if (g.epi != kEpiBf16Add) prefetch_tmap(&tma_out);
   }
   if (warp == 1) {
     tmem_alloc(tmem_base_slot, kTmemCols);
@@ -196,14 +219,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
 
-  auto tile_coords = [&](int tile, int& mb, int& nb) {
+  // tile -> (m block, n block, K split); K splits vary slowest
+  auto tile_coords = [&](int tile, int& mb, int& nb, int& ks) {
+    const int per = g.tiles_m * g.tiles_n;
+    ks = tile / per;
+    const int t = tile - ks * per;
     if (g.m_fastest) {
-      mb = tile % g.tiles_m;
-      nb = tile / g.tiles_m;
+      mb = t % g.tiles_m;
+      nb = t / g.tiles_m;
     } else {
-      nb = tile % g.tiles_n;
-      mb = tile / g.tiles_n;
+      nb = t % g.tiles_n;
+      mb = t / g.tiles_n;
     }
+  };
+  auto kb_range = [&](int ks, int& kb0, int& kb1) {
+    kb0 = ks * g.kb_per_split;
+    kb1 = min(g.num_kb, kb0 + g.kb_per_split);
   };
 
   if (warp == 0) {
@@ -213,10 +244,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool run = true;
       for (int tile = blockIdx.x; tile < num_tiles && run; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, mb, nb);
+        int mb, nb, ks, kb0, kb1;
+        tile_coords(tile, mb, nb, ks);
+        kb_range(ks, kb0, kb1);
         const int m0 = mb * kBM, n0 = nb * kBN;
-        for (int kb = 0; kb < g.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(&empty[stage], phase ^ 1, abort_flag)) {
             run = false;
             break;
@@ -254,10 +286,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       bool run = true;
       for (int tile = blockIdx.x; tile < num_tiles && run; tile += gridDim.x) {
+        int mb, nb, ks, kb0, kb1;
+        tile_coords(tile, mb, nb, ks);
+        kb_range(ks, kb0, kb1);
         if (!wait_or_abort(&tmem_empty[acc], acc_phase ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
-        for (int kb = 0; kb < g.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_or_abort(&full[stage], phase, abort_flag)) {
             run = false;
             break;
@@ -271,7 +306,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // M/N-major: it moves 16 rows (2 x 1024-byte swizzle atoms).
             const uint64_t ad = A_MN ? smem_desc(sa + k * 2048, 8192, 1024) : smem_desc(sa + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);  // stage free once these MMAs have read it
           if (++stage == kStages) {
@@ -289,69 +324,106 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int r_local = q * 32 + lane;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access: rows 32q .. 32q + 31
+    uint8_t* my_stage = out_stage + q * 2 * kStageOutBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
+    int nstore = 0;  // bulk groups committed by this warp (lane 0)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      int mb, nb;
-      tile_coords(tile, mb, nb);
+      int mb, nb, ks;
+      tile_coords(tile, mb, nb, ks);
       if (!wait_or_abort(&tmem_full[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
-      const int row = mb * kBM + r_local;
-      const bool row_ok = row < g.m_limit;
       const uint32_t t_row = tmem_base + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
+      const int y = ks * g.split_rows + mb * kBM + q * 32;  // first output row of this warp
+      if (g.epi == kEpiStoreBf16) {
+        // 64-column slices: 2 TMEM loads -> 32 rows x 128 bytes, 128-byte swizzled
 #pragma unroll 1
-      for (int cc = 0; cc < kBN; cc += 32) {
-        uint32_t v[32];
-        tmem_ld32(t_row + cc, v);
-        tmem_ld_wait();
-        const int col0 = nb * kBN + cc;
-        if (!row_ok || col0 >= g.n_limit) continue;
-        const int ncols = min(32, g.n_limit - col0);  // a multiple of 8
-        if (g.epi == kEpiStoreBf16 || g.epi == kEpiBf16Add) {
+        for (int cs = 0; cs < kBN; cs += 64) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(t_row + cs, v0);
+          tmem_ld32(t_row + cs + 32, v1);
+          tmem_ld_wait();
+          uint8_t* buf = my_stage + (nstore & 1) * kStageOutBytes;
+          if (nstore >= 2) {
+            if (lane == 0) bulk_wait_read_1();
+            __syncwarp();
+          }
+          uint8_t* rowp = buf + lane * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* src = c < 4 ? &v0[c * 8] : &v1[(c - 4) * 8];
+            const uint4 w = make_uint4(
+                pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+                pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+                pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+                pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) = w;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_out, buf, nb * kBN + cs, y);
+            bulk_commit();
+          }
+          ++nstore;
+        }
+      } else if (g.epi == kEpiStoreF32 || g.epi == kEpiAddF32) {
+        // 32-column slices: 1 TMEM load -> 32 rows x 128 bytes of fp32
+#pragma unroll 1
+        for (int cs = 0; cs < kBN; cs += 32) {
+          uint32_t v[32];
+          tmem_ld32(t_row + cs, v);
+          tmem_ld_wait();
+          uint8_t* buf = my_stage + (nstore & 1) * kStageOutBytes;
+          if (nstore >= 2) {
+            if (lane == 0) bulk_wait_read_1();
+            __syncwarp();
+          }
+          uint8_t* rowp = buf + lane * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(v[c * 4], v[c * 4 + 1], v[c * 4 + 2], v[c * 4 + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (g.epi == kEpiStoreF32) tma_store_2d(&tma_out, buf, nb * kBN + cs, y);
+            else tma_reduce_add_2d(&tma_out, buf, nb * kBN + cs, y);
+            bulk_commit();
+          }
+          ++nstore;
+        }
+      } else {
+        // kEpiBf16Add: accumulate into the bf16 output with plain loads and stores
+        const int row = mb * kBM + q * 32 + lane;
+        const bool row_ok = row < g.m_limit;
+#pragma unroll 1
+        for (int cc = 0; cc < kBN; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(t_row + cc, v);
+          tmem_ld_wait();
+          const int col0 = nb * kBN + cc;
+          if (!row_ok || col0 >= g.n_limit) continue;
+          const int ncols = min(32, g.n_limit - col0);  // a multiple of 8
           uint16_t* o = reinterpret_cast<uint16_t*>(g.out) + static_cast<int64_t>(row) * g.ld_out + col0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (j * 8 >= ncols) break;
+            const uint4 prev = *reinterpret_cast<const uint4*>(o + j * 8);
             float f[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[j * 8 + e]);
-            if (g.epi == kEpiBf16Add) {
-              const uint4 prev = *reinterpret_cast<const uint4*>(o + j * 8);
-              f[0] += bf16_lo(prev.x); f[1] += bf16_hi(prev.x);
-              f[2] += bf16_lo(prev.y); f[3] += bf16_hi(prev.y);
-              f[4] += bf16_lo(prev.z); f[5] += bf16_hi(prev.z);
-              f[6] += bf16_lo(prev.w); f[7] += bf16_hi(prev.w);
-            }
+            f[0] += bf16_lo(prev.x); f[1] += bf16_hi(prev.x);
+            f[2] += bf16_lo(prev.y); f[3] += bf16_hi(prev.y);
+            f[4] += bf16_lo(prev.z); f[5] += bf16_hi(prev.z);
+            f[6] += bf16_lo(prev.w); f[7] += bf16_hi(prev.w);
             *reinterpret_cast<uint4*>(o + j * 8) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                                                               pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
           }
-        } else {
-          float* a = g.acc + static_cast<int64_t>(row) * g.ld_acc + col0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j * 8 >= ncols) break;
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[j * 8 + e]);
-            if (g.epi != kEpiAccWrite) {
-              const float4 p0 = *reinterpret_cast<const float4*>(a + j * 8);
-              const float4 p1 = *reinterpret_cast<const float4*>(a + j * 8 + 4);
-              f[0] += p0.x; f[1] += p0.y; f[2] += p0.z; f[3] += p0.w;
-              f[4] += p1.x; f[5] += p1.y; f[6] += p1.z; f[7] += p1.w;
-            }
-            if (g.epi == kEpiAccFinal) {
-              uint16_t* o = reinterpret_cast<uint16_t*>(g.out) + static_cast<int64_t>(row) * g.ld_out + col0;
-              *reinterpret_cast<uint4*>(o + j * 8) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-            } else {
-              *reinterpret_cast<float4*>(a + j * 8) = make_float4(f[0], f[1], f[2], f[3]);
-              *reinterpret_cast<float4*>(a + j * 8 + 4) = make_float4(f[4], f[5], f[6], f[7]);
-            }
-          }
         }
       }
+      // every TMEM load of this accumulator is complete: hand it back to the MMA warp
       tc_fence_before();
       mbar_arrive(&tmem_empty[acc]);
       if (++acc == 2) {
@@ -359,6 +431,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1;
       }
     }
+    if (lane == 0) bulk_wait_all();  // staging buffers stay valid until the stores have read them
   }
 
   // ---------------- teardown ----------------

@@ -8,9 +8,12 @@
 //                                     by the valid-token count of the whole call
 //   3  dX_c   = G_c W                 tcgen05 GEMM (A K-major, B N-major)
 //   4  dW    (+)= G_c^T X_c           tcgen05 GEMM (both operands M/N-major);
-//                                     fp32 accumulator across chunks, cast once
-//                                     by the last chunk's epilogue ("fp32"), or
-//                                     accumulated in the bf16 output ("weight")
+//                                     fp32 accumulator across chunks (TMA store,
+//                                     then TMA reduce-add in L2), rounded once to
+//                                     bf16 at the end ("fp32"), or accumulated in
+//                                     the bf16 output ("weight")
+// When the dX tiles alone would leave SMs idle, dX splits K into fp32 partials
+// that a second kernel sums in a fixed order (deterministic).
 //
 // The loss is the fixed-order sum of all rows' losses, divided by the valid
 // count for "mean".  ld = round_up(V, 8) keeps chunk rows 16-byte aligned as
@@ -43,19 +46,53 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows of
-// `row_bytes`, box {64, box_outer}, 128-byte swizzle, zero fill outside.
+// 2-D tensor map: `inner` contiguous elements per row, `outer` rows of
+// `row_bytes`, box {box_inner, box_outer}, 128-byte swizzle, zero fill
+// outside (loads) / clipping (stores).
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-               uint32_t box_outer) {
+               uint32_t box_outer, bool f32 = false, uint32_t box_inner = 64) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {64, box_outer};
+  const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output maps of the GEMM epilogue: 32-row boxes of 128 bytes (64 bf16 or 32 fp32).
+bool make_out_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld) {
+  return make_tmap(m, base, cols, rows, ld * 2, 32, false, 64);
+}
+bool make_out_f32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld) {
+  return make_tmap(m, base, cols, rows, ld * 4, 32, true, 32);
+}
+
+// out[r, c] = bf16(sum_s ws[s][r, c]) for r < rows, in split order (deterministic).
+__global__ void splitk_reduce_kernel(const float* __restrict__ ws, int splits, int64_t split_stride, int rows,
+                                     int cols, uint16_t* __restrict__ out, int64_t ld_out) {
+  const int64_t n4 = static_cast<int64_t>(rows) * (cols / 4);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / (cols / 4), c4 = i - r * (cols / 4);
+    float4 a = *reinterpret_cast<const float4*>(ws + r * cols + 4 * c4);
+    for (int sp = 1; sp < splits; ++sp) {
+      const float4 b = *reinterpret_cast<const float4*>(ws + sp * split_stride + r * cols + 4 * c4);
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    *reinterpret_cast<uint2*>(out + r * ld_out + 4 * c4) = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+}
+
+// out = bf16(acc), the fp32 weight-gradient accumulator's single final rounding.
+__global__ void cast_bf16_kernel(const float* __restrict__ acc, int64_t n4, uint16_t* __restrict__ out) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[i];
+    reinterpret_cast<uint2*>(out)[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
 }
 
 int sm_count() {
@@ -66,8 +103,8 @@ int sm_count() {
 }
 
 template <bool A_MN, bool B_MN>
-gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const sm100::GemmArgs& g, int kind,
-                        cudaStream_t stream) {
+gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
+                        const sm100::GemmArgs& g, int kind, cudaStream_t stream) {
   auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -75,13 +112,51 @@ gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const sm10
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm100::kGemmSmem);
   });
   if (attr_err != cudaSuccess) return GH_ERR_CUDA;
-  const int tiles = g.tiles_m * g.tiles_n;
+  const int tiles = g.tiles_m * g.tiles_n * g.k_splits;
   if (tiles == 0) return GH_OK;
   const int grid = std::min(tiles, sm_count());
   ProfileScope prof(kind, stream);
-  kern<<<grid, sm100::kGemmThreads, sm100::kGemmSmem, stream>>>(ta, tb, g);
+  kern<<<grid, sm100::kGemmThreads, sm100::kGemmSmem, stream>>>(ta, tb, tout, g);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+}
+
+sm100::GemmArgs gemm_args(int M, int N, int K, int m_fastest, int epi) {
+  sm100::GemmArgs g{};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.tiles_m = (M + sm100::kBM - 1) / sm100::kBM;
+  g.tiles_n = (N + sm100::kBN - 1) / sm100::kBN;
+  g.num_kb = (K + sm100::kBK - 1) / sm100::kBK;
+  g.k_splits = 1;
+  g.kb_per_split = g.num_kb;
+  g.m_fastest = m_fastest;
+  g.epi = epi;
+  g.m_limit = M;
+  g.n_limit = N;
+  return g;
+}
+
+// K splits for a GEMM whose output tiles would leave SMs idle: the split count
+// that minimises (waves of work units) x (K steps per unit), each unit at
+// least 16 K steps long; the smallest such count on ties.
+int choose_splits(int tiles, int num_kb, int sms) {
+  if (tiles >= sms) return 1;
+  int best = 1;
+  int64_t best_cost = static_cast<int64_t>(num_kb);
+  const int smax = std::max(1, num_kb / 16);
+  for (int sp = 2; sp <= smax; ++sp) {
+    const int per = (num_kb + sp - 1) / sp;
+    const int used = (num_kb + per - 1) / per;
+    const int64_t waves = (static_cast<int64_t>(tiles) * used + sms - 1) / sms;
+    const int64_t cost = waves * per;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = used;
+    }
+  }
+  return best;
 }
 
 int64_t default_chunk(int64_t N, int64_t ld) {
@@ -107,13 +182,22 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const int64_t nchunks = (N + chunk - 1) / chunk;
   if (chunk > INT32_MAX / 2 || V > INT32_MAX / 2) return GH_ERR_UNSUPPORTED;
   const bool acc32 = a.accum == GH_ACCUM_FP32 && nchunks > 1;
+  const int sms = sm_count();
+  const int tiles_m_max = static_cast<int>((chunk + sm100::kBM - 1) / sm100::kBM);
+  const int dx_num_kb = static_cast<int>((V + sm100::kBK - 1) / sm100::kBK);
+  const int dx_tiles_max = tiles_m_max * static_cast<int>((D + sm100::kBN - 1) / sm100::kBN);
+  const int dx_splits = choose_splits(dx_tiles_max, dx_num_kb, sms);
+  const int64_t rows_pad = static_cast<int64_t>(tiles_m_max) * sm100::kBM;
 
-  // scratch: [counter | row losses | chunk buffer | fp32 accumulator]
+  // scratch: [counter | row losses | chunk buffer | fp32 dW accumulator | dX split partials]
   const size_t off_rows = 256;
   const size_t off_buf = (off_rows + sizeof(float) * N + 255) / 256 * 256;
   const size_t buf_bytes = static_cast<size_t>(chunk) * ld * 2;
   const size_t off_acc = (off_buf + buf_bytes + 255) / 256 * 256;
-  const size_t total = off_acc + (acc32 ? static_cast<size_t>(V) * D * 4 : 0);
+  const size_t acc_bytes = acc32 ? static_cast<size_t>(V) * D * 4 : 0;
+  const size_t off_ws = (off_acc + acc_bytes + 255) / 256 * 256;
+  const size_t ws_bytes = dx_splits > 1 ? static_cast<size_t>(dx_splits) * rows_pad * D * 4 : 0;
+  const size_t total = off_ws + ws_bytes;
   void* scratch = nullptr;
   gh_status_t st = scratch_alloc(&scratch, total, stream);
   if (st != GH_OK) return st;
@@ -122,6 +206,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   float* row_loss = reinterpret_cast<float*>(base + off_rows);
   uint16_t* L = reinterpret_cast<uint16_t*>(base + off_buf);
   float* acc = acc32 ? reinterpret_cast<float*>(base + off_acc) : nullptr;
+  float* ws = dx_splits > 1 ? reinterpret_cast<float*>(base + off_ws) : nullptr;
 
   const uint16_t* X = static_cast<const uint16_t*>(a.X);
   const uint16_t* W = static_cast<const uint16_t*>(a.W);
@@ -129,9 +214,13 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   uint16_t* dW = static_cast<uint16_t*>(a.dW);
 
   st = ce_count_launch(a.targets, N, V, a.ignore_index, n_valid, stream);
-  // W as the K-major B operand of the logits GEMM and the N-major B operand of dX.
-  CUtensorMap tm_w_k, tm_w_n;
-  if (st == GH_OK && (!make_tmap(&tm_w_k, W, D, V, D * 2, sm100::kBN) || !make_tmap(&tm_w_n, W, D, V, D * 2, 64)))
+  // W as the K-major B operand of the logits GEMM and the N-major B operand of
+  // dX; the weight-gradient output (bf16) and accumulator (fp32) maps.
+  CUtensorMap tm_w_k, tm_w_n, tm_dw_out, tm_acc, tm_ws;
+  if (st == GH_OK &&
+      (!make_tmap(&tm_w_k, W, D, V, D * 2, sm100::kBN) || !make_tmap(&tm_w_n, W, D, V, D * 2, 64) ||
+       !make_out_bf16(&tm_dw_out, dW, D, V, D) || (acc32 && !make_out_f32(&tm_acc, acc, D, V, D)) ||
+       (ws && !make_out_f32(&tm_ws, ws, D, dx_splits * rows_pad, D))))
     st = GH_ERR_CUDA;
 
   for (int64_t c = 0; c < nchunks && st == GH_OK; ++c) {
@@ -139,23 +228,17 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     const int rows = static_cast<int>(std::min<int64_t>(chunk, N - c0));
     const uint16_t* Xc = X + c0 * D;
 
-    // 1: L = X_c W^T
-    CUtensorMap tm_x_k, tm_l_k, tm_l_m, tm_x_n;
+    CUtensorMap tm_x_k, tm_l_k, tm_l_m, tm_x_n, tm_l_out, tm_dx_out;
     if (!make_tmap(&tm_x_k, Xc, D, rows, D * 2, sm100::kBM) || !make_tmap(&tm_l_k, L, V, rows, ld * 2, sm100::kBM) ||
-        !make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) || !make_tmap(&tm_x_n, Xc, D, rows, D * 2, 64)) {
+        !make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) || !make_tmap(&tm_x_n, Xc, D, rows, D * 2, 64) ||
+        !make_out_bf16(&tm_l_out, L, V, rows, ld) || !make_out_bf16(&tm_dx_out, dX + c0 * D, D, rows, D)) {
       st = GH_ERR_CUDA;
       break;
     }
-    sm100::GemmArgs g1{};
-    g1.M = rows; g1.N = static_cast<int>(V); g1.K = static_cast<int>(D);
-    g1.tiles_m = (rows + sm100::kBM - 1) / sm100::kBM;
-    g1.tiles_n = static_cast<int>((V + sm100::kBN - 1) / sm100::kBN);
-    g1.num_kb = static_cast<int>((D + sm100::kBK - 1) / sm100::kBK);
-    g1.m_fastest = 1;
-    g1.epi = sm100::kEpiStoreBf16;
-    g1.out = L; g1.ld_out = ld;
-    g1.m_limit = rows; g1.n_limit = static_cast<int>(ld);
-    st = launch_gemm<false, false>(tm_x_k, tm_w_k, g1, GH_KERNEL_LOGITS_GEMM, stream);
+
+    // 1: L = X_c W^T
+    sm100::GemmArgs g1 = gemm_args(rows, static_cast<int>(V), static_cast<int>(D), 1, sm100::kEpiStoreBf16);
+    st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, GH_KERNEL_LOGITS_GEMM, stream);
     if (st != GH_OK) break;
 
     // 2: per-row loss and the logits gradient, in place
@@ -175,38 +258,50 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     st = ce_launch(ca, rows, GH_BF16, stream);
     if (st != GH_OK) break;
 
-    // 3: dX_c = G_c W
-    sm100::GemmArgs g3{};
-    g3.M = rows; g3.N = static_cast<int>(D); g3.K = static_cast<int>(V);
-    g3.tiles_m = (rows + sm100::kBM - 1) / sm100::kBM;
-    g3.tiles_n = static_cast<int>((D + sm100::kBN - 1) / sm100::kBN);
-    g3.num_kb = static_cast<int>((V + sm100::kBK - 1) / sm100::kBK);
-    g3.m_fastest = 1;
-    g3.epi = sm100::kEpiStoreBf16;
-    g3.out = dX + c0 * D; g3.ld_out = D;
-    g3.m_limit = rows; g3.n_limit = static_cast<int>(D);
-    st = launch_gemm<false, true>(tm_l_k, tm_w_n, g3, GH_KERNEL_DX_GEMM, stream);
-    if (st != GH_OK) break;
+    // 3: dX_c = G_c W (K split into fp32 partials when the tiles alone leave SMs idle)
+    sm100::GemmArgs g3 = gemm_args(rows, static_cast<int>(D), static_cast<int>(V), 1, sm100::kEpiStoreBf16);
+    const int splits = choose_splits(g3.tiles_m * g3.tiles_n, g3.num_kb, sms);
+    if (splits > 1 && ws) {
+      g3.k_splits = std::min(splits, dx_splits);
+      g3.kb_per_split = (g3.num_kb + g3.k_splits - 1) / g3.k_splits;
+      g3.k_splits = (g3.num_kb + g3.kb_per_split - 1) / g3.kb_per_split;
+      g3.split_rows = static_cast<int>(rows_pad);
+      g3.epi = sm100::kEpiStoreF32;
+      st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_ws, g3, GH_KERNEL_DX_GEMM, stream);
+      if (st != GH_OK) break;
+      splitk_reduce_kernel<<<sms * 4, 256, 0, stream>>>(ws, g3.k_splits, rows_pad * D, rows, static_cast<int>(D),
+                                                        dX + c0 * D, D);
+      note_launch();
+      if (cudaGetLastError() != cudaSuccess) {
+        st = GH_ERR_CUDA;
+        break;
+      }
+    } else {
+      st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_dx_out, g3, GH_KERNEL_DX_GEMM, stream);
+      if (st != GH_OK) break;
+    }
 
     // 4: dW (+)= G_c^T X_c
-    sm100::GemmArgs g4{};
-    g4.M = static_cast<int>(V); g4.N = static_cast<int>(D); g4.K = rows;
-    g4.tiles_m = static_cast<int>((V + sm100::kBM - 1) / sm100::kBM);
-    g4.tiles_n = static_cast<int>((D + sm100::kBN - 1) / sm100::kBN);
-    g4.num_kb = (rows + sm100::kBK - 1) / sm100::kBK;
-    g4.m_fastest = 0;
-    g4.out = dW; g4.ld_out = D;
-    g4.acc = acc; g4.ld_acc = D;
-    g4.m_limit = static_cast<int>(V); g4.n_limit = static_cast<int>(D);
+    sm100::GemmArgs g4 = gemm_args(static_cast<int>(V), static_cast<int>(D), rows, 0, sm100::kEpiStoreBf16);
+    g4.out = dW;
+    g4.ld_out = D;
+    const CUtensorMap* out4 = &tm_dw_out;
     if (a.accum == GH_ACCUM_FP32) {
-      if (nchunks == 1) g4.epi = sm100::kEpiStoreBf16;
-      else if (c == 0) g4.epi = sm100::kEpiAccWrite;
-      else if (c + 1 < nchunks) g4.epi = sm100::kEpiAccAdd;
-      else g4.epi = sm100::kEpiAccFinal;
+      if (acc32) {
+        g4.epi = c == 0 ? sm100::kEpiStoreF32 : sm100::kEpiAddF32;
+        out4 = &tm_acc;
+      }
     } else {
       g4.epi = c == 0 ? sm100::kEpiStoreBf16 : sm100::kEpiBf16Add;
     }
-    st = launch_gemm<true, true>(tm_l_m, tm_x_n, g4, GH_KERNEL_DW_GEMM, stream);
+    st = launch_gemm<true, true>(tm_l_m, tm_x_n, *out4, g4, GH_KERNEL_DW_GEMM, stream);
+  }
+  if (st == GH_OK && acc32) {
+    // the fp32 accumulator's single rounding to the weight dtype
+    const int64_t n4 = V * D / 4;
+    cast_bf16_kernel<<<sms * 4, 256, 0, stream>>>(acc, n4, dW);
+    note_launch();
+    if (cudaGetLastError() != cudaSuccess) st = GH_ERR_CUDA;
   }
   if (st == GH_OK) st = ce_reduce_launch(row_loss, N, n_valid, a.mean, a.loss, stream);
   scratch_free(scratch, stream);
