@@ -24,6 +24,8 @@
 #include <cstdlib>
 #include <mutex>
 
+#include <cuda_fp16.h>
+
 #include "ce.h"
 #include "common.cuh"
 #include "profile.h"
@@ -206,11 +208,9 @@ __device__ __forceinline__ uint4 pack_f16x8(const float (&e)[N]) {  // fp32 rows
 }
 
 __device__ __forceinline__ float2 f16x2_to_f32(uint32_t w) {
-  float lo, hi;
-  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(w));
-  return make_float2(lo, hi);
+  __half2 h;
+  memcpy(&h, &w, sizeof(h));
+  return __half22float2(h);
 }
 
 __device__ __forceinline__ float f16_to_f32(uint16_t h) {
@@ -226,18 +226,26 @@ __device__ __forceinline__ void unpack_f16x8(const uint4& q, float (&g)[N]) {
   if constexpr (N == 8) { g[4] = c.x; g[5] = c.y; g[6] = d.x; g[7] = d.y; }
 }
 
-constexpr int kRowThreads = 512;
+#ifndef GH_CE_ROW_THREADS
+#define GH_CE_ROW_THREADS 512
+#endif
+constexpr int kRowThreads = GH_CE_ROW_THREADS;  // two row groups of half this size
+#ifndef GH_CE_UNROLL
+#define GH_CE_UNROLL 4
+#endif
+constexpr int kUnroll = GH_CE_UNROLL;  // chunks a thread handles per loop iteration
 constexpr int kStreamThreads = 1024;
 constexpr int kPieces = 4;                     // bulk copies (and barriers) per slice
 constexpr int kMinPieceChunks = 256;           // 4 KiB
-constexpr int kHdrBytes = 384;                 // barriers, targets, records, reduction scratch
+constexpr int kHdrBytes = 1024;                // barriers, targets, records, reduction scratch
 constexpr int kMaxSliceBytes = 110 * 1024;     // two slice buffers per CTA fit in 227 KiB
+constexpr int kMaxCluster = 8;
 
 struct RowShared {
-  uint64_t full[2][kPieces];                   // load barriers of the two buffer slots
+  uint64_t full[2][kPieces];                   // load barriers of the two groups' buffers
+  uint64_t xbar[2][2];                         // per group, per valid-row parity: cluster records in
   int64_t tgt[2][2];                           // per group: targets of its next two rows
-  float rec_m[2], rec_s[2], rec_xt[2];         // partials published to the cluster,
-  int rec_has_t[2];                            //   double-buffered by valid-row parity
+  float4 xrec[2][2][kMaxCluster];              // per group, per parity, per rank: (m, s, xt, has_t)
   float lse[2], xt[2], xt_local[2];            // per group, broadcast within the group
   float pad_[2];
   float red_m[kRowThreads / 32];
@@ -282,24 +290,24 @@ __device__ __forceinline__ bool target_valid(const CeArgs& a, int64_t t) {
   return (t != a.ignore_index) && t >= 0 && t < a.V;
 }
 
-__device__ __forceinline__ int npieces_of(int nbulk) {
-  return nbulk == 0 ? 0 : max(1, min(kPieces, nbulk / kMinPieceChunks));
-}
 
-// Group leader: start the bulk copies of this CTA's slice of `row` into `buf`
-// (one per piece, each on its own barrier).
+// Group leader: start the bulk copies of this CTA's slice of `row` into `buf`.
+// Every valid row arrives on all a.npieces barriers of the buffer (the piece
+// count is fixed per launch, so the barriers' phases stay in step however the
+// rows' alignment varies); a piece with no bytes completes on the arrive alone.
 template <int ES>
 __device__ __forceinline__ void issue_slice(const CeArgs& a, int64_t row, int64_t t, int rank, uint8_t* buf,
                                             uint64_t* bars) {
   if (row >= a.B || !target_valid(a, t)) return;
   const SliceGeo g = slice_geo<ES>(a, row, rank);
   const int nb = g.x_hi - g.x_lo;
-  const int np = npieces_of(nb);
+  const int np = a.npieces;
   const uint8_t* gbase = g.gsrc - g.lead;
   for (int p = 0; p < np; ++p) {
     const int cs = g.x_lo + (nb * p) / np, ce = g.x_lo + (nb * (p + 1)) / np;
-    mbar_arrive_expect_tx(&bars[p], 16u * (ce - cs));
-    bulk_g2s(buf + 16 * cs, gbase + 16 * cs, 16u * (ce - cs), &bars[p]);
+    const uint32_t bytes = 16u * (ce - cs);
+    mbar_arrive_expect_tx(&bars[p], bytes);
+    if (bytes) bulk_g2s(buf + 16 * cs, gbase + 16 * cs, bytes, &bars[p]);
   }
 }
 
@@ -369,13 +377,13 @@ __global__ void __launch_bounds__(1024) ce_count1_kernel(const int64_t* __restri
 //      owner afterwards with the -scale term.
 // fp32 rows only sum in pass 1 and re-evaluate the exponent in pass 2 (a
 // cache would not fit in place).
-template <typename T, int NG>
+template <typename T>
 __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
+  constexpr int NG = 2;                 // row groups per CTA
   constexpr int ES = Elem<T>::kBytes;
   constexpr int EPC = 16 / ES;
   constexpr int NT = kRowThreads / NG;  // threads per group
   constexpr int GW = NT / 32;           // warps per group
-  constexpr int L = NG == 1 ? 2 : 1;    // rows in flight per group (buffers)
   constexpr bool kBf16 = ES == 2;
   constexpr float kShift = kBf16 ? 14.0f : 0.0f;  // log2 of the fp16 cache scale
   extern __shared__ __align__(128) uint8_t smem[];
@@ -389,18 +397,18 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
   const int rank = blockIdx.x - cid * S;
   const int64_t ngroups = static_cast<int64_t>(gridDim.x / S) * NG;
   const int64_t first = static_cast<int64_t>(cid) * NG + grp;
-  auto gsync = [&]() {
-    if constexpr (NG == 1) __syncthreads();
-    else asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(NT) : "memory");
-  };
-  auto slot_of = [&](int64_t k) { return NG == 1 ? static_cast<int>(k & 1) : grp; };
+  auto gsync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(NT) : "memory"); };
+  auto slot_of = [&](int64_t) { return grp; };
   auto buf_of = [&](int slot) { return smem + kHdrBytes + slot * a.buf_bytes; };
   auto row_of = [&](int64_t k) { return first + k * ngroups; };
   auto tgt_of = [&](int64_t k) { return row_of(k) < a.B ? a.targets[row_of(k)] : int64_t(0); };
 
   if (threadIdx.x == 0) {
-    for (int sl = 0; sl < 2; ++sl)
+    for (int sl = 0; sl < 2; ++sl) {
       for (int p = 0; p < kPieces; ++p) mbar_init(&sh.full[sl][p], 1);
+      mbar_init(&sh.xbar[sl][0], S);
+      mbar_init(&sh.xbar[sl][1], S);
+    }
     fence_mbar_init();
   }
   if (leader) {
@@ -408,12 +416,15 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
     sh.tgt[grp][1] = tgt_of(1);
   }
   __syncthreads();
-  if (leader)
-    for (int64_t k = 0; k < L; ++k) issue_slice<ES>(a, row_of(k), sh.tgt[grp][k & 1], rank, buf_of(slot_of(k)),
-                                                    sh.full[slot_of(k)]);
+  if (S > 1) {  // every CTA's exchange barriers are initialised before any peer arrives on them
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  }
+  if (leader) issue_slice<ES>(a, row_of(0), sh.tgt[grp][0], rank, buf_of(grp), sh.full[grp]);
 
   uint32_t phase = 0;       // bit sl: parity of the next waits on slot sl
-  uint32_t valid_rows = 0;  // selects the cluster record buffer
+  uint32_t valid_rows = 0;  // selects the exchange barrier and record buffer
+  uint32_t xphase = 0;      // bit pb: parity of the next wait on xbar[grp][pb]
   bool ok = true;
   const unsigned long long nv = *a.n_valid;
   const float scale = a.mean ? 1.0f / static_cast<float>(nv > 0 ? nv : 1ull) : 1.0f;
@@ -442,7 +453,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
     } else {
       // ---- pass 0: this thread's max, piece by piece as copies land ----------------------
       const int nb = g.x_hi - g.x_lo;
-      const int np = npieces_of(nb);
+      const int np = a.npieces;
       // ragged ends outside the bulk range: element loads by their owners
       auto fill_edge = [&](int c) {
         for (int bb = 16 * c; bb < 16 * c + 16; bb += ES) {
@@ -480,18 +491,24 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
         if (p == np - 1 && g.x_hi == g.nchunks && (g.span & 15) && tid == (g.nchunks - 1) % NT)
           for (int bb = g.span; bb < 16 * g.nchunks; bb += ES) *reinterpret_cast<T*>(buf + bb) = neg_inf_elem<T>();
         int c = cs + ((tid - cs) % NT + NT) % NT;
-        for (; c + NT < ce; c += 2 * NT) {
-          fold_max(c);
-          if constexpr (kBf16) {
-            const uint4 q = *reinterpret_cast<const uint4*>(buf + 16 * (c + NT));
-            mx1 = bf16x2_max(mx1, bf16x2_max(bf16x2_max(q.x, q.y), bf16x2_max(q.z, q.w)));
-          } else {
-            fold_max(c + NT);
+        for (; c + (kUnroll - 1) * NT < ce; c += kUnroll * NT) {
+          uint4 q[kUnroll];
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) q[u] = *reinterpret_cast<const uint4*>(buf + 16 * (c + u * NT));
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            if constexpr (kBf16) {
+              uint32_t& m = (u & 1) ? mx1 : mx0;
+              m = bf16x2_max(m, bf16x2_max(bf16x2_max(q[u].x, q[u].y), bf16x2_max(q[u].z, q[u].w)));
+            } else {
+              mf = fmaxf(mf, fmaxf(fmaxf(__uint_as_float(q[u].x), __uint_as_float(q[u].y)),
+                                   fmaxf(__uint_as_float(q[u].z), __uint_as_float(q[u].w))));
+            }
           }
         }
-        if (c < ce) fold_max(c);
+        for (; c < ce; c += NT) fold_max(c);
       }
-      if (np > 0) phase ^= 1u << sl;
+      phase ^= 1u << sl;  // every valid row completes one phase on each piece barrier
       float m_t;
       if constexpr (kBf16) {
         mx0 = bf16x2_max(mx0, mx1);
@@ -526,19 +543,18 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
           for (int j = 0; j < EPC; j += 2) acc = __fadd2_rn(acc, make_float2(e[j], e[j + 1]));
         };
         int c = tid;
-        for (; c + NT < g.nchunks; c += 2 * NT) {
-          uint4* p0 = reinterpret_cast<uint4*>(buf + 16 * c);
-          uint4* p1 = reinterpret_cast<uint4*>(buf + 16 * (c + NT));
-          const uint4 q0 = *p0, q1 = *p1;
-          float e0[EPC], e1[EPC];
-          exps(q0, e0);
-          exps(q1, e1);
-          if constexpr (kBf16) {
-            *p0 = pack_f16x8(e0);
-            *p1 = pack_f16x8(e1);
+        for (; c + (kUnroll - 1) * NT < g.nchunks; c += kUnroll * NT) {
+          uint4 q[kUnroll];
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) q[u] = *reinterpret_cast<const uint4*>(buf + 16 * (c + u * NT));
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            float e[EPC];
+            exps(q[u], e);
+            if constexpr (kBf16) *reinterpret_cast<uint4*>(buf + 16 * (c + u * NT)) = pack_f16x8(e);
           }
         }
-        if (c < g.nchunks) {
+        for (; c < g.nchunks; c += NT) {
           uint4* p0 = reinterpret_cast<uint4*>(buf + 16 * c);
           float e0[EPC];
           exps(*p0, e0);
@@ -561,7 +577,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
         red_s[gwarp] = ms.s;
       }
       gsync();
-      const int rb = valid_rows & 1;
+      const int pb = valid_rows & 1;
       if (gwarp == 0) {
         MaxSum w = lane < GW ? MaxSum{red_m[lane], red_s[lane]} : MaxSum{kNegInf, 0.0f};
 #pragma unroll
@@ -575,31 +591,29 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
             sh.lse[grp] = w.m + logf(s_cta);
             sh.xt[grp] = sh.xt_local[grp];
           } else {
-            sh.rec_m[rb] = w.m;
-            sh.rec_s[rb] = s_cta;
-            sh.rec_has_t[rb] = has_t ? 1 : 0;
-            sh.rec_xt[rb] = has_t ? sh.xt_local[grp] : 0.0f;
-            fence_cluster();  // the record is visible cluster-wide before this thread arrives
-          }
-        }
-      }
-      if constexpr (NG == 1) {
-        if (S > 1) {
-          cluster_arrive_relaxed();
-          cluster_wait_acquire();
-          if (leader) {
+            // Publish this slice's (max, sum, target logit) into every rank's
+            // record slot `rank` and arrive on its barrier for this row parity;
+            // then wait for all ranks' records here and combine them in rank
+            // order (the same lse on every CTA).
+            const float xtv = has_t ? sh.xt_local[grp] : 0.0f;
+            for (int q = 0; q < S; ++q) {
+              st_dsmem_v4(map_to_rank(&sh.xrec[grp][pb][rank], q), w.m, s_cta, xtv, has_t ? 1.0f : 0.0f);
+              mbar_arrive_cluster(map_to_rank(&sh.xbar[grp][pb], q));
+            }
+            if (!mbar_wait_cluster(&sh.xbar[grp][pb], (xphase >> pb) & 1)) ok = false;
             MaxSum tot{kNegInf, 0.0f};
             float x = 0.0f;
-            for (int r = 0; r < S; ++r) {  // fixed rank order: identical on every CTA
-              MaxSum pr{ld_dsmem_f32(map_to_rank(&sh.rec_m[rb], r)), ld_dsmem_f32(map_to_rank(&sh.rec_s[rb], r))};
-              tot = combine(tot, pr);
-              if (ld_dsmem_s32(map_to_rank(&sh.rec_has_t[rb], r))) x = ld_dsmem_f32(map_to_rank(&sh.rec_xt[rb], r));
+            for (int q = 0; q < S; ++q) {
+              const float4 r = sh.xrec[grp][pb][q];
+              tot = combine(tot, MaxSum{r.x, r.y});
+              if (r.w != 0.0f) x = r.z;
             }
-            sh.lse[0] = tot.m + logf(tot.s);
-            sh.xt[0] = x;
+            sh.lse[grp] = tot.m + logf(tot.s);
+            sh.xt[grp] = x;
           }
         }
       }
+      if (S > 1) xphase ^= 1u << pb;
       gsync();
       const float lse = sh.lse[grp];
       ++valid_rows;
@@ -638,16 +652,18 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
         if (a.congruent) {
           uint8_t* dbase = g.gdst - g.lead;
           int c = g.c_lo + ((tid - g.c_lo) % NT + NT) % NT;
-          for (; c + NT < g.c_hi; c += 2 * NT) {
-            const uint4 q0 = *reinterpret_cast<const uint4*>(buf + 16 * c);
-            const uint4 q1 = *reinterpret_cast<const uint4*>(buf + 16 * (c + NT));
-            float g0[EPC], g1[EPC];
-            grad16(q0, g0);
-            grad16(q1, g1);
-            *reinterpret_cast<uint4*>(dbase + 16 * c) = pack16<T>(g0);
-            *reinterpret_cast<uint4*>(dbase + 16 * (c + NT)) = pack16<T>(g1);
+          for (; c + (kUnroll - 1) * NT < g.c_hi; c += kUnroll * NT) {
+            uint4 q[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) q[u] = *reinterpret_cast<const uint4*>(buf + 16 * (c + u * NT));
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+              float g0[EPC];
+              grad16(q[u], g0);
+              *reinterpret_cast<uint4*>(dbase + 16 * (c + u * NT)) = pack16<T>(g0);
+            }
           }
-          if (c < g.c_hi) {
+          for (; c < g.c_hi; c += NT) {
             const uint4 q0 = *reinterpret_cast<const uint4*>(buf + 16 * c);
             float g0[EPC];
             grad16(q0, g0);
@@ -687,16 +703,11 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
     gsync();
     if (leader) {
       sh.tgt[grp][k & 1] = t_ahead;  // row k + 2's target (row k + 1's is already stored)
-      const int64_t kn = k + L;      // next row into this slot
-      issue_slice<ES>(a, row_of(kn), L == 2 ? t_ahead : sh.tgt[grp][kn & 1], rank, buf, sh.full[sl]);
+      issue_slice<ES>(a, row_of(k + 1), sh.tgt[grp][(k + 1) & 1], rank, buf, sh.full[sl]);
     }
   }
-  if constexpr (NG == 1) {
-    if (S > 1) {  // no CTA leaves while a peer may still read its records
-      cluster_arrive_relaxed();
-      cluster_wait_acquire();
-    }
-  }
+  // No peer writes into this CTA after its last row: every rank's last records
+  // for this CTA were waited for above.
 }
 
 // Rows too long for the shared-memory path: one CTA per row, two passes over
@@ -819,7 +830,7 @@ CePlan ce_plan(int64_t V, int elem_bytes) {
     return ((q + 15) / 16) * 16;  // slices start on 32/64-byte boundaries of the row
   };
   int S = 1;
-  while (S < 8 && slice_for(S) * elem_bytes > target) S *= 2;
+  while (S < kMaxCluster && slice_for(S) * elem_bytes > target) ++S;
   const int64_t q = slice_for(S);
   if (q * elem_bytes > kMaxSliceBytes) {
     p.streaming = true;
@@ -844,12 +855,7 @@ static int device_sm_count() {
 
 namespace {
 
-// Rows of one slice run two row groups per CTA; rows split over a cluster run
-// one double-buffered group.
-void (*row_kernel_for(int es, int cluster))(CeArgs) {
-  if (es == 4) return cluster == 1 ? ce_row_kernel<float, 2> : ce_row_kernel<float, 1>;
-  return cluster == 1 ? ce_row_kernel<uint16_t, 2> : ce_row_kernel<uint16_t, 1>;
-}
+void (*row_kernel_for(int es))(CeArgs) { return es == 4 ? ce_row_kernel<float> : ce_row_kernel<uint16_t>; }
 
 // Launch plan of the row kernel for one (device, V, element size), computed
 // once: the occupancy queries and attribute calls cost far more than a launch.
@@ -879,17 +885,17 @@ gh_status_t row_plan(int64_t V, int es, CePlan* out, int64_t* active_out) {
   const CePlan plan = ce_plan(V, es);
   int64_t active = 0;
   if (!plan.streaming) {
-    void (*kern)(CeArgs) = row_kernel_for(es, plan.cluster);
+    void (*kern)(CeArgs) = row_kernel_for(es);
     // The dynamic shared memory limit is an attribute of the kernel, shared by
     // every plan: raise it once per device to the opt-in maximum.
-    static bool raised[64][2][2] = {};
-    const int kv = es == 4, kg = plan.cluster == 1;
-    if (dev < 64 && !raised[dev][kv][kg]) {
+    static bool raised[64][2] = {};
+    const int kv = es == 4;
+    if (dev < 64 && !raised[dev][kv]) {
       int optin = 0;
       if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return GH_ERR_CUDA;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
         return GH_ERR_CUDA;
-      raised[dev][kv][kg] = true;
+      raised[dev][kv] = true;
     }
     if (plan.smem_bytes > kHdrBytes + 2 * (kMaxSliceBytes + 256)) return GH_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
@@ -934,6 +940,7 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
   a.cluster = plan.cluster;
   a.slice = plan.slice;
   a.buf_bytes = plan.buf_bytes;
+  a.npieces = std::max(1, std::min(kPieces, (plan.slice * es / 16) / kMinPieceChunks));
 
   if (plan.streaming) {
     if (B > INT32_MAX) return GH_ERR_UNSUPPORTED;
@@ -944,7 +951,7 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
     return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
   }
 
-  void (*kern)(CeArgs) = row_kernel_for(es, plan.cluster);
+  void (*kern)(CeArgs) = row_kernel_for(es);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kRowThreads);
   cfg.dynamicSmemBytes = plan.smem_bytes;
@@ -957,9 +964,8 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // Persistent grid: as many clusters as can be resident at once, no more
-  // than there are rows (two per CTA with two row groups).
-  const int64_t per_cluster = plan.cluster == 1 ? 2 : 1;
-  const int64_t nclusters = std::min<int64_t>(active, (B + per_cluster - 1) / per_cluster);
+  // than there are rows (two per cluster, one per row group).
+  const int64_t nclusters = std::min<int64_t>(active, (B + 1) / 2);
   cfg.gridDim = dim3(static_cast<unsigned>(nclusters * plan.cluster));
   ProfileScope prof(a.profile_kind, stream);
   note_launch();

@@ -23,6 +23,7 @@ struct CeArgs {
   int slice;                          // elements per CTA (set by ce_launch)
   int cluster;                        // CTAs per row (set by ce_launch)
   int buf_bytes;                      // bytes per slice buffer (set by ce_launch)
+  int npieces;                        // bulk copies per slice (set by ce_launch)
   int congruent;                      // (logits - grad) % 16 == 0
   int profile_kind;                   // gh_kernel_t the row kernel is timed as
 };

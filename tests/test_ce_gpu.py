@@ -58,7 +58,9 @@ def test_cluster_paths(cuda_device, dtype, V, B):
 
 
 @pytest.mark.parametrize("dtype,V,B", [("bf16", 5003, 1500), ("f32", 30011, 700), ("bf16", 100003, 700),
-                                       ("bf16", 262147, 300)])
+                                       ("bf16", 262147, 300),
+                                       # slices whose chunk count straddles 1024 from row to row
+                                       ("bf16", 8187, 1500), ("f32", 4093, 1500)])
 def test_many_rows_per_persistent_cta(cuda_device, dtype, V, B):
     # more rows than resident CTAs: each CTA cycles both slice buffers many
     # times, with ignored rows (no copy, no cluster exchange) interleaved
