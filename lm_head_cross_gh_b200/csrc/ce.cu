@@ -315,6 +315,8 @@ __device__ __forceinline__ void issue_slice(const CeArgs& a, int64_t row, int64_
 
 __global__ void ce_count_kernel(const int64_t* __restrict__ t, int64_t n, int64_t V, int64_t ii,
                                 unsigned long long* __restrict__ count) {
+  pdl_wait();
+  pdl_trigger();
   unsigned long long c = 0;
   bool bad = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
@@ -334,6 +336,8 @@ __global__ void ce_count_kernel(const int64_t* __restrict__ t, int64_t n, int64_
 __global__ void __launch_bounds__(1024) ce_count1_kernel(const int64_t* __restrict__ t, int64_t n, int64_t V,
                                                          int64_t ii, unsigned long long* __restrict__ count) {
   __shared__ unsigned long long part[32];
+  pdl_wait();
+  pdl_trigger();
   unsigned long long c = 0;
   bool bad = false;
   for (int64_t i = threadIdx.x; i < n; i += 1024) {
@@ -411,6 +415,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
     }
     fence_mbar_init();
   }
+  pdl_wait();     // the predecessor's outputs (targets, logits, counter) are complete
+  pdl_trigger();  // persistent grid: every CTA is resident, the next kernel may start launching
   if (leader) {
     sh.tgt[grp][0] = tgt_of(0);
     sh.tgt[grp][1] = tgt_of(1);
@@ -717,6 +723,7 @@ __global__ void __launch_bounds__(kStreamThreads) ce_stream_kernel(CeArgs a) {
   constexpr int ES = Elem<T>::kBytes;
   constexpr int EPC = 16 / ES;
   __shared__ float red[2 * (kStreamThreads / 32)];
+  pdl_wait();
   const int tid = threadIdx.x;
   const int64_t row = blockIdx.x;
   const int64_t V = a.V;
@@ -791,6 +798,8 @@ __global__ void __launch_bounds__(1024) ce_reduce_kernel(const float* __restrict
                                                          const unsigned long long* __restrict__ n_valid,
                                                          int mean, float* __restrict__ loss) {
   __shared__ double red[32];
+  pdl_wait();
+  pdl_trigger();
   double s = 0.0;
   for (int64_t i = threadIdx.x; i < B; i += 1024) s += static_cast<double>(row_loss[i]);
 #pragma unroll
@@ -822,16 +831,11 @@ static int ce_slice_target_bytes() {
   return v;
 }
 
-CePlan ce_plan(int64_t V, int elem_bytes) {
+// Plan for rows of V elements split over a cluster of S CTAs.
+static CePlan plan_for_cluster(int64_t V, int elem_bytes, int S) {
   CePlan p{};
-  const int64_t target = ce_slice_target_bytes();
-  auto slice_for = [&](int s) {
-    const int64_t q = (V + s - 1) / s;
-    return ((q + 15) / 16) * 16;  // slices start on 32/64-byte boundaries of the row
-  };
-  int S = 1;
-  while (S < kMaxCluster && slice_for(S) * elem_bytes > target) ++S;
-  const int64_t q = slice_for(S);
+  int64_t q = (V + S - 1) / S;
+  q = ((q + 15) / 16) * 16;  // slices start on 32/64-byte boundaries of the row
   if (q * elem_bytes > kMaxSliceBytes) {
     p.streaming = true;
     p.cluster = 1;
@@ -844,6 +848,15 @@ CePlan ce_plan(int64_t V, int elem_bytes) {
   p.buf_bytes = static_cast<int>(((16 * chunks) + 127) / 128 * 128);
   p.smem_bytes = kHdrBytes + 2 * p.buf_bytes;
   return p;
+}
+
+// The smallest cluster whose slices fit the slice target (a launch may still
+// pick a larger one that keeps more SMs busy: see row_plan).
+CePlan ce_plan(int64_t V, int elem_bytes) {
+  const int64_t target = ce_slice_target_bytes();
+  int S = 1;
+  while (S < kMaxCluster && ((V + S - 1) / S + 15) / 16 * 16 * elem_bytes > target) ++S;
+  return plan_for_cluster(V, elem_bytes, S);
 }
 
 static int device_sm_count() {
@@ -882,7 +895,7 @@ gh_status_t row_plan(int64_t V, int es, CePlan* out, int64_t* active_out) {
       return GH_OK;
     }
   }
-  const CePlan plan = ce_plan(V, es);
+  CePlan plan = ce_plan(V, es);
   int64_t active = 0;
   if (!plan.streaming) {
     void (*kern)(CeArgs) = row_kernel_for(es);
@@ -897,24 +910,30 @@ gh_status_t row_plan(int64_t V, int es, CePlan* out, int64_t* active_out) {
         return GH_ERR_CUDA;
       raised[dev][kv] = true;
     }
+    // Clusters must fit inside a GPC, so the number resident at once depends on
+    // the cluster size.  (A larger cluster that keeps more SMs busy measured
+    // slower: 262144-vocab rows, 6 CTAs x 22 clusters 1.22 ms vs 5 x 26 1.11 ms.)
+    auto resident = [&](const CePlan& pl) -> int64_t {
+      cudaLaunchConfig_t cfg = {};
+      cfg.blockDim = dim3(kRowThreads);
+      cfg.dynamicSmemBytes = pl.smem_bytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = pl.cluster;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      cfg.gridDim = dim3(static_cast<unsigned>(pl.cluster * device_sm_count()));
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+      }
+      return n;
+    };
+    active = resident(plan);
     if (plan.smem_bytes > kHdrBytes + 2 * (kMaxSliceBytes + 256)) return GH_ERR_UNSUPPORTED;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kRowThreads);
-    cfg.dynamicSmemBytes = plan.smem_bytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = plan.cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cfg.gridDim = dim3(static_cast<unsigned>(plan.cluster * device_sm_count()));
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-      (void)cudaGetLastError();
-      n = 0;
-    }
-    active = n;
     if (active <= 0) return GH_ERR_UNSUPPORTED;
   }
   if (std::getenv("GH_DEBUG_PLAN"))
@@ -945,31 +964,24 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
   if (plan.streaming) {
     if (B > INT32_MAX) return GH_ERR_UNSUPPORTED;
     ProfileScope prof(a.profile_kind, stream);
-    if (dtype == GH_F32) ce_stream_kernel<float><<<static_cast<unsigned>(B), kStreamThreads, 0, stream>>>(a);
-    else ce_stream_kernel<uint16_t><<<static_cast<unsigned>(B), kStreamThreads, 0, stream>>>(a);
+    const cudaError_t e = dtype == GH_F32
+                              ? launch_pdl(ce_stream_kernel<float>, dim3(static_cast<unsigned>(B)), dim3(kStreamThreads),
+                                           0, stream, 1, a)
+                              : launch_pdl(ce_stream_kernel<uint16_t>, dim3(static_cast<unsigned>(B)),
+                                           dim3(kStreamThreads), 0, stream, 1, a);
     note_launch();
-    return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+    return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
   }
 
   void (*kern)(CeArgs) = row_kernel_for(es);
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kRowThreads);
-  cfg.dynamicSmemBytes = plan.smem_bytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = plan.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   // Persistent grid: as many clusters as can be resident at once, no more
   // than there are rows (two per cluster, one per row group).
   const int64_t nclusters = std::min<int64_t>(active, (B + 1) / 2);
-  cfg.gridDim = dim3(static_cast<unsigned>(nclusters * plan.cluster));
   ProfileScope prof(a.profile_kind, stream);
   note_launch();
-  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return GH_ERR_CUDA;
+  if (launch_pdl(kern, dim3(static_cast<unsigned>(nclusters * plan.cluster)), dim3(kRowThreads), plan.smem_bytes,
+                 stream, plan.cluster, a) != cudaSuccess)
+    return GH_ERR_CUDA;
   return GH_OK;
 }
 
@@ -977,22 +989,23 @@ gh_status_t ce_count_launch(const int64_t* targets, int64_t n, int64_t V, int64_
                             unsigned long long* count, cudaStream_t stream) {
   if (n <= (int64_t(1) << 20)) {
     // one CTA counts without atomics and writes the counter itself
-    ce_count1_kernel<<<1, 1024, 0, stream>>>(targets, n, V, ii, count);
+    const cudaError_t e = launch_pdl(ce_count1_kernel, dim3(1), dim3(1024), 0, stream, 1, targets, n, V, ii, count);
     note_launch();
-    return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+    return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
   }
   if (cudaMemsetAsync(count, 0, sizeof(unsigned long long), stream) != cudaSuccess) return GH_ERR_CUDA;
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 4);
-  ce_count_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(targets, n, V, ii, count);
+  const cudaError_t e =
+      launch_pdl(ce_count_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, 1, targets, n, V, ii, count);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+  return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
 }
 
 gh_status_t ce_reduce_launch(const float* row_loss, int64_t B, const unsigned long long* n_valid, int mean,
                              float* loss, cudaStream_t stream) {
-  ce_reduce_kernel<<<1, 1024, 0, stream>>>(row_loss, B, n_valid, mean, loss);
+  const cudaError_t e = launch_pdl(ce_reduce_kernel, dim3(1), dim3(1024), 0, stream, 1, row_loss, B, n_valid, mean, loss);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+  return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
 }
 
 }  // namespace gh

@@ -218,6 +218,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
+  pdl_wait();     // operands and outputs are free of the predecessor kernel from here on
+  pdl_trigger();  // one CTA per SM, all resident: the next kernel may start its prologue
 
   // tile -> (m block, n block, K split); K splits vary slowest
   auto tile_coords = [&](int tile, int& mb, int& nb, int& ks) {

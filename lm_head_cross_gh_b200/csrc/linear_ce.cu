@@ -73,6 +73,8 @@ bool make_out_f32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows
 // out[r, c] = bf16(sum_s ws[s][r, c]) for r < rows, in split order (deterministic).
 __global__ void splitk_reduce_kernel(const float* __restrict__ ws, int splits, int64_t split_stride, int rows,
                                      int cols, uint16_t* __restrict__ out, int64_t ld_out) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t n4 = static_cast<int64_t>(rows) * (cols / 4);
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -88,6 +90,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ ws, int splits, i
 
 // out = bf16(acc), the fp32 weight-gradient accumulator's single final rounding.
 __global__ void cast_bf16_kernel(const float* __restrict__ acc, int64_t n4, uint16_t* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float4 a = reinterpret_cast<const float4*>(acc)[i];
@@ -116,9 +120,10 @@ gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
   if (tiles == 0) return GH_OK;
   const int grid = std::min(tiles, sm_count());
   ProfileScope prof(kind, stream);
-  kern<<<grid, sm100::kGemmThreads, sm100::kGemmSmem, stream>>>(ta, tb, tout, g);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(sm100::kGemmThreads), sm100::kGemmSmem, stream, 1, ta, tb,
+                                   tout, g);
   note_launch();
-  return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+  return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
 }
 
 sm100::GemmArgs gemm_args(int M, int N, int K, int m_fastest, int epi) {
@@ -269,10 +274,11 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       g3.epi = sm100::kEpiStoreF32;
       st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_ws, g3, GH_KERNEL_DX_GEMM, stream);
       if (st != GH_OK) break;
-      splitk_reduce_kernel<<<sms * 4, 256, 0, stream>>>(ws, g3.k_splits, rows_pad * D, rows, static_cast<int>(D),
-                                                        dX + c0 * D, D);
+      const cudaError_t e = launch_pdl(splitk_reduce_kernel, dim3(sms * 4), dim3(256), 0, stream, 1,
+                                       static_cast<const float*>(ws), g3.k_splits, rows_pad * D, rows,
+                                       static_cast<int>(D), dX + c0 * D, D);
       note_launch();
-      if (cudaGetLastError() != cudaSuccess) {
+      if (e != cudaSuccess) {
         st = GH_ERR_CUDA;
         break;
       }
@@ -299,9 +305,10 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   if (st == GH_OK && acc32) {
     // the fp32 accumulator's single rounding to the weight dtype
     const int64_t n4 = V * D / 4;
-    cast_bf16_kernel<<<sms * 4, 256, 0, stream>>>(acc, n4, dW);
+    const cudaError_t e =
+        launch_pdl(cast_bf16_kernel, dim3(sms * 4), dim3(256), 0, stream, 1, static_cast<const float*>(acc), n4, dW);
     note_launch();
-    if (cudaGetLastError() != cudaSuccess) st = GH_ERR_CUDA;
+    if (e != cudaSuccess) st = GH_ERR_CUDA;
   }
   if (st == GH_OK) st = ce_reduce_launch(row_loss, N, n_valid, a.mean, a.loss, stream);
   scratch_free(scratch, stream);
