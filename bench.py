@@ -148,11 +148,14 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 
 class Dist:
+    """One process per GPU (torchrun env vars); NCCL on GPUs, gloo on CPU (tests)."""
+
     def __init__(self):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = False
+        self.backend = None
 
     def init(self, backend="nccl"):
         if self.world > 1:
@@ -161,35 +164,48 @@ class Dist:
             os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
             self.pg = True
+            self.backend = backend
+
+    def _device(self):
+        return "cuda" if self.backend == "nccl" else "cpu"
 
     def barrier(self):
         if self.pg:
             import torch
             import torch.distributed as dist
-            dist.barrier(device_ids=[torch.cuda.current_device()]) if dist.get_backend() == "nccl" else dist.barrier()
+            if self.backend == "nccl":
+                dist.barrier(device_ids=[torch.cuda.current_device()])
+            else:
+                dist.barrier()
+
+    def _reduce(self, v: float, op) -> float:
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=self._device())
+        dist.all_reduce(t, op=op)
+        return float(t.item())
 
     def max(self, v: float) -> float:
-        if not self.pg:
-            return v
-        import torch
         import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return self._reduce(v, dist.ReduceOp.MAX) if self.pg else v
 
     def sum(self, v: float) -> float:
-        if not self.pg:
-            return v
-        import torch
         import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+        return self._reduce(v, dist.ReduceOp.SUM) if self.pg else v
 
     def close(self):
         if self.pg:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+def aggregate(dist, ms_local: float, tokens_local: float):
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    ms = dist.max(ms_local)
+    tokens = dist.sum(tokens_local)
+    return tokens / (ms * 1e-3), ms
 
 
 # --------------------------------------------------------------------------
@@ -229,62 +245,108 @@ def pinned(a):
     return t.pin_memory()
 
 
+CE_OPS = ("fwd_bwd", "fwd", "select")
+
+
+def select_index(targets):
+    """selective_log_softmax has no ignore_index: ignored targets select class 0."""
+    import numpy as np
+    return np.ascontiguousarray(np.maximum(targets, 0))
+
+
+def ce_config(p, op):
+    return {"workload": p.name, "op": op, "B": p.B, "V": p.V, "dtype": p.dtype, "reduction": p.reduction,
+            "z_loss": p.z_loss, "ignore_index": p.ignore_index,
+            "ignored_rows": int((p.targets == p.ignore_index).sum()),
+            "l2": f"inputs larger than L2 ({p.B * p.V * (4 if p.dtype == 'f32' else 2) / 1e6:.0f} MB); no flush"}
+
+
+def ce_oracle_rows(p, op, rows):
+    """The float64 oracle on a sample of rows, for the operation `op`."""
+    import numpy as np
+    import oracle
+    x = p.values_f32(rows).astype(np.float64)
+    if op == "select":
+        oracle.selective_log_softmax(x, select_index(p.targets[rows]))
+    else:
+        _, scale = oracle.n_valid_and_scale(p.targets, p.ignore_index, p.reduction, p.V)
+        oracle.ce_rows(x, p.targets[rows], p.ignore_index, p.z_loss, scale, with_grad=op == "fwd_bwd")
+    return len(rows)
+
+
 class CeCase:
+    """Standalone CE on one batch: forward+backward (gh_ce_fwd_bwd), the loss
+    alone (gh_ce_fwd) or the selected log-probabilities (gh_selective_log_softmax)."""
     kind = "ce"
 
-    def __init__(self, name, seed, dev):
-        import numpy as np
+    def __init__(self, name, seed, dev, op="fwd_bwd"):
         import torch
+        self.op = op
         self.p = make_ce(name, seed)
-        self.h_x = pinned(self.p.logits)
-        self.h_t = pinned(self.p.targets)
+        p = self.p
+        self.h_x = pinned(p.logits)
+        self.h_t = pinned(select_index(p.targets) if op == "select" else p.targets)
         self.x = self.h_x.to(dev, non_blocking=False)
         self.t = self.h_t.to(dev)
-        self.grad = torch.empty_like(self.x)
+        self.grad = torch.empty_like(self.x) if op == "fwd_bwd" else None
         self.loss = torch.empty((), dtype=torch.float32, device=dev)
         self.h_loss = torch.empty((), dtype=torch.float32).pin_memory()
-        self.tokens = self.p.B
-        es = 4 if self.p.dtype == "f32" else 2
-        n_ign = int((self.p.targets == self.p.ignore_index).sum())
-        # algorithmic bytes: read every valid row once, write every gradient row once, read targets
-        self.bytes_per_step = ((self.p.B - n_ign) * self.p.V + self.p.B * self.p.V) * es + 8 * self.p.B
+        self.sel = torch.empty(p.B, dtype=torch.float32, device=dev) if op == "select" else None
+        self.h_sel = torch.empty(p.B, dtype=torch.float32).pin_memory() if op == "select" else None
+        self.tokens = p.B
+        es = 4 if p.dtype == "f32" else 2
+        n_ign = int((p.targets == p.ignore_index).sum())
+        # algorithmic bytes: every row the operation reads once (ignored rows are
+        # not read by the losses), every gradient row written once, the targets,
+        # and the selected values written
+        if op == "fwd_bwd":
+            self.bytes_per_step = ((p.B - n_ign) * p.V + p.B * p.V) * es + 8 * p.B
+        elif op == "fwd":
+            self.bytes_per_step = (p.B - n_ign) * p.V * es + 8 * p.B
+        else:
+            self.bytes_per_step = p.B * p.V * es + 12 * p.B
         self.h2d = self.h_x.numel() * self.h_x.element_size() + self.h_t.numel() * 8
-        self.d2h = 4
-        self.dtype = "bf16" if self.p.dtype == "bf16" else "f32"
+        self.d2h = 4 * p.B if op == "select" else 4
+        self.dtype = "bf16" if p.dtype == "bf16" else "f32"
+
+    def _call(self):
+        import lm_head_cross_gh_b200 as gh
+        p = self.p
+        if self.op == "fwd_bwd":
+            gh.gh_ce_fwd_bwd(self.x, self.t, p.ignore_index, p.reduction, p.z_loss, grad=self.grad, loss=self.loss)
+        elif self.op == "fwd":
+            gh.gh_ce_fwd(self.x, self.t, p.ignore_index, p.reduction, p.z_loss, loss=self.loss)
+        else:
+            gh.gh_selective_log_softmax(self.x, self.t, out=self.sel)
 
     def step(self):
-        import lm_head_cross_gh_b200 as gh
-        p = self.p
-        gh.gh_ce_fwd_bwd(self.x, self.t, p.ignore_index, p.reduction, p.z_loss, grad=self.grad, loss=self.loss)
+        self._call()
 
     def e2e_step(self):
-        import lm_head_cross_gh_b200 as gh
-        p = self.p
         self.x.copy_(self.h_x, non_blocking=True)
         self.t.copy_(self.h_t, non_blocking=True)
-        gh.gh_ce_fwd_bwd(self.x, self.t, p.ignore_index, p.reduction, p.z_loss, grad=self.grad, loss=self.loss)
-        self.h_loss.copy_(self.loss, non_blocking=True)
+        self._call()
+        if self.op == "select":
+            self.h_sel.copy_(self.sel, non_blocking=True)
+        else:
+            self.h_loss.copy_(self.loss, non_blocking=True)
 
     def config(self):
-        p = self.p
-        return {"workload": p.name, "B": p.B, "V": p.V, "dtype": p.dtype, "reduction": p.reduction,
-                "z_loss": p.z_loss, "ignore_index": p.ignore_index,
-                "ignored_rows": int((p.targets == p.ignore_index).sum()),
-                "l2": f"inputs larger than L2 ({p.B * p.V * (4 if p.dtype == 'f32' else 2) / 1e6:.0f} MB); no flush"}
+        return ce_config(self.p, self.op)
 
     def cpu_sample(self, budget_rows):
         import numpy as np
-        p = self.p
-        rows = np.arange(min(p.B, budget_rows))
-        return rows
+        return np.arange(min(self.p.B, budget_rows))
 
     def run_oracle(self, rows):
-        import numpy as np
-        import oracle
-        p = self.p
-        _, scale = oracle.n_valid_and_scale(p.targets, p.ignore_index, p.reduction, p.V)
-        oracle.ce_rows(p.values_f32(rows).astype(np.float64), p.targets[rows], p.ignore_index, p.z_loss, scale)
-        return len(rows)
+        return ce_oracle_rows(self.p, self.op, rows)
+
+
+def linear_config(p):
+    return {"workload": p.name, "N": p.N, "D": p.D, "V": p.V, "chunk": p.chunk, "accum": p.accum,
+            "reduction": p.reduction, "z_loss": p.z_loss,
+            "ignored_rows": int((p.targets == p.ignore_index).sum()),
+            "l2": "weight and chunk logits larger than L2; no flush"}
 
 
 class LinearCase:
@@ -327,11 +389,7 @@ class LinearCase:
         self.h_loss.copy_(self.loss, non_blocking=True)
 
     def config(self):
-        p = self.p
-        return {"workload": p.name, "N": p.N, "D": p.D, "V": p.V, "chunk": p.chunk, "accum": p.accum,
-                "reduction": p.reduction, "z_loss": p.z_loss,
-                "ignored_rows": int((p.targets == p.ignore_index).sum()),
-                "l2": "weight and chunk logits larger than L2; no flush"}
+        return linear_config(self.p)
 
     def cpu_sample(self, budget_rows):
         import numpy as np
@@ -465,10 +523,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="ce_gpt2", choices=list(CE_WORKLOADS) + list(LINEAR_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--op", default="fwd_bwd", choices=list(CE_OPS),
+                    help="standalone CE operation timed on a CE workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-linear", action="store_true", help="omit the linear-CE object on the CE line")
     ap.add_argument("--rows", type=int, default=0, help="use only the first ROWS rows/tokens (profiling cases)")
+    ap.add_argument("--launches-only", action="store_true",
+                    help="run W + K steps and exit without timing or report (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -490,25 +552,29 @@ def main():
     pk, pk_kind = peaks()
 
     is_ce = args.workload in CE_WORKLOADS
-    case = CeCase(args.workload, dist.rank, dev) if is_ce else LinearCase(args.workload, dist.rank, dev)
+    case = CeCase(args.workload, dist.rank, dev, args.op) if is_ce else LinearCase(args.workload, dist.rank, dev)
+    if args.launches_only:
+        for _ in range(args.warmup + args.steps):
+            case.step()
+        torch.cuda.synchronize()
+        dist.close()
+        return 0
     clocks = ClockSampler(dist.local)
     ms, launches, kern = time_steps(case, dist, args.steps, args.warmup, clocks)
-    ms_max = dist.max(ms)
-    tokens_all = dist.sum(case.tokens * args.steps)
-    value = tokens_all / (ms_max * 1e-3)
+    value, ms_max = aggregate(dist, ms, case.tokens * args.steps)
 
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": case.dtype,
            "data": "synthetic (seeded; seed = rank)", "config": case.config()}
-    out["config"]["parallelism"] = f"replicas x{dist.world} (independent batches, no collective)"
+    out["config"]["parallelism"] = parallelism(dist.world)
 
     if is_ce:
         k_ms, k_n = kern["ce_row"]
         k_avg = k_ms / max(k_n, 1)
         achieved = case.bytes_per_step / (k_avg * 1e-3) / 1e9
         digest = source_digest(["lm_head_cross_gh_b200/csrc/ce.cu", "lm_head_cross_gh_b200/csrc/common.cuh"])
-        traffic = profiled_traffic("ce_row_kernel.md", digest, case.p.name)
+        traffic = profiled_traffic("ce_row_kernel.md", digest, case.p.name) if case.op == "fwd_bwd" else None
         out["roofline"] = {"bound": "hbm", "kernel": "ce_row_kernel", "achieved": achieved,
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                            "traffic": traffic, "algorithmic_bytes": case.bytes_per_step,
@@ -567,6 +633,10 @@ def linear_roofline(case, kern, steps, pk, pk_kind):
             "peak_source": f"{pk_kind} bf16 (sustained)"}
 
 
+def parallelism(world):
+    return f"replicas x{world} (independent batches, no collective)"
+
+
 def reference_arm(args, dist):
     """The float64 oracle on the host cores, on a bounded sample of the same workload."""
     if dist.rank != 0:
@@ -575,18 +645,18 @@ def reference_arm(args, dist):
 
     class Dummy:
         pass
+    case = Dummy()
     if is_ce:
-        case = Dummy()
         case.p = make_ce(args.workload, 0)
-        case.kind = "ce"
         case.cpu_sample = lambda n, c=case: __import__("numpy").arange(min(c.p.B, n))
-        case.run_oracle = lambda rows, c=case: CeCase.run_oracle(c, rows)
+        case.run_oracle = lambda rows, c=case: ce_oracle_rows(c.p, args.op, rows)
+        config = ce_config(case.p, args.op)
     else:
-        case = Dummy()
         case.p = make_linear(args.workload, 0)
-        case.kind = "linear"
         case.cpu_sample = lambda n, c=case: __import__("numpy").arange(min(c.p.N, n))
         case.run_oracle = lambda rows, c=case: LinearCase.run_oracle(c, rows)
+        config = linear_config(case.p)
+    config["parallelism"] = parallelism(1)
     rows_per_step = max(1, ORACLE_ROWS[args.workload] // 8)
     rows = case.cpu_sample(rows_per_step)
     for _ in range(args.warmup):
@@ -601,7 +671,7 @@ def reference_arm(args, dist):
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-           "dtype": "f64", "data": "synthetic (seeded)", "config": {"workload": case.p.name},
+           "dtype": "f64", "data": "synthetic (seeded)", "config": config,
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)

@@ -1,14 +1,17 @@
 /*
  * gh.h — C ABI of libgh, next-token cross-entropy for NVIDIA B200 (sm_100a).
  *
- * Two operations, both from the Greyhound functional API
- * (greyhound.nn.functional):
+ * Operations from the Greyhound functional API (greyhound.nn.functional):
  *
  *  - gh_ce_fwd_bwd: `cross_entropy` — materialised [B, V] logits and [B]
  *    targets; the summed (or mean) loss with optional z-loss and the logits
- *    gradient "in one streaming pass".  nuvec FastOp::CrossEntropy gives the
- *    row loss logsumexp(x) - x[target] (float32) and FastOp::CrossEntropyVjp
- *    its logits gradient.
+ *    gradient, both from one pass that streams each row.  nuvec
+ *    FastOp::CrossEntropy gives the row loss logsumexp(x) - x[target]
+ *    (float32) and FastOp::CrossEntropyVjp its logits gradient.
+ *  - gh_ce_fwd: the same loss without the gradient (evaluation; Gpt2 `loss`,
+ *    viv `gpt_loss`), optionally unreduced.
+ *  - gh_selective_log_softmax: `selective_log_softmax` — one log-probability
+ *    per row, x[index] - logsumexp(x), without the full log-softmax.
  *  - gh_linear_ce: `chunked_linear_cross_entropy` — logits = inputs @ weight.T
  *    computed one row chunk at a time and never materialised in full; per
  *    chunk the logits gradient G gives grad_inputs[chunk] = G @ weight and
@@ -126,6 +129,39 @@ gh_status_t gh_ce_fwd_bwd_noalloc(const void* logits, const int64_t* targets, in
                                   float z_mult, float* loss, void* grad, void* stream);
 
 /*
+ * gh_ce_fwd — the cross-entropy loss of gh_ce_fwd_bwd without its gradient:
+ * the evaluation form (a forward with no tape and no gradients), reading the
+ * logits once.
+ *
+ *   logits, targets, B, V, dtype, ignore_index, reduction, z_mult, loss
+ *            as for gh_ce_fwd_bwd.
+ *   row_loss optional device float32 [B] (NULL: not returned); written with
+ *            each row's loss before reduction, 0 for ignored rows (the
+ *            unreduced loss).
+ * Scratch (stream-ordered): 16 bytes, plus 4*B bytes when row_loss is NULL.
+ */
+gh_status_t gh_ce_fwd(const void* logits, const int64_t* targets, int64_t B, int64_t V,
+                      gh_dtype_t dtype, int64_t ignore_index, gh_reduction_t reduction,
+                      float z_mult, float* loss, float* row_loss, void* stream);
+
+/*
+ * gh_selective_log_softmax — Greyhound `selective_log_softmax`: for each row
+ * r, out[r] = x[r, index[r]] - logsumexp(x[r, :]), the log-probability of one
+ * selected class, without materialising the log-probabilities.
+ *
+ *   logits   [rows, V] of `dtype` (GH_F32 or GH_BF16), device (any leading
+ *            shape flattened to rows).
+ *   index    [rows] int64, device.
+ *   rows >= 0, V >= 1 (V < 2^31).
+ *   out      [rows] float32, device, written.
+ * No ignore_index: every row is computed.  An index outside [0, V) violates
+ * the precondition: that row's logits are not read, out[r] = NaN, and
+ * GH_ERR_TARGET_RANGE is recorded in the device status word.  No scratch.
+ */
+gh_status_t gh_selective_log_softmax(const void* logits, const int64_t* index, int64_t rows, int64_t V,
+                                     gh_dtype_t dtype, float* out, void* stream);
+
+/*
  * gh_linear_ce — chunked fused linear cross-entropy (Greyhound
  * `chunked_linear_cross_entropy` over `chunked_linear_loss`).
  *
@@ -160,7 +196,8 @@ gh_status_t gh_get_device_status(void* stream);
 /*
  * Kernel timing (for benchmarks and roofline reports).  Kernel kinds: */
 typedef enum {
-  GH_KERNEL_CE_ROW = 0,        /* standalone CE row kernel (one per gh_ce_fwd_bwd) */
+  GH_KERNEL_CE_ROW = 0,        /* standalone CE row kernel (one per gh_ce_fwd_bwd, gh_ce_fwd,
+                                  gh_selective_log_softmax) */
   GH_KERNEL_LOGITS_GEMM = 1,   /* linear-CE: chunk logits = X_c @ W^T (+ CE epilogue) */
   GH_KERNEL_CHUNK_CE = 2,      /* linear-CE: per-chunk loss and logits gradient */
   GH_KERNEL_DX_GEMM = 3,       /* linear-CE: grad_inputs[chunk] = G_c @ W */

@@ -63,6 +63,11 @@ def lib() -> ctypes.CDLL:
     L.gh_ce_fwd_bwd.restype = c_int
     L.gh_ce_fwd_bwd_noalloc.argtypes = list(L.gh_ce_fwd_bwd.argtypes)
     L.gh_ce_fwd_bwd_noalloc.restype = c_int
+    L.gh_ce_fwd.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_int, c_float,
+                            c_void_p, c_void_p, c_void_p]
+    L.gh_ce_fwd.restype = c_int
+    L.gh_selective_log_softmax.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_void_p, c_void_p]
+    L.gh_selective_log_softmax.restype = c_int
     L.gh_linear_ce.argtypes = [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int,
                                c_int64, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p]
     L.gh_linear_ce.restype = c_int
@@ -182,6 +187,62 @@ def gh_ce_fwd_bwd_noalloc(logits, targets, ignore_index: int = -100, reduction: 
                                      _stream_handle(stream))
     _check(st, "gh_ce_fwd_bwd_noalloc")
     return loss, grad
+
+
+def gh_ce_fwd(logits, targets, ignore_index: int = -100, reduction: str = "mean", z_loss: float = 0.0, *,
+              loss=None, row_loss=None, stream=None):
+    """Cross-entropy loss without the gradient (one call into ``gh_ce_fwd``).
+
+    ``logits`` CUDA [B, V] float32 or bfloat16, ``targets`` CUDA int64 [B].
+    ``row_loss`` (optional float32 [B] output) receives each row's loss
+    (0 for ignored rows), the unreduced form.  Returns ``(loss, row_loss)``;
+    ``row_loss`` is None unless it was given.
+    """
+    import torch
+    _need(logits.dim() == 2 and logits.is_cuda and logits.is_contiguous(), "logits: contiguous CUDA [B, V]")
+    _need(logits.dtype in (torch.float32, torch.bfloat16), "logits dtype must be float32 or bfloat16")
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
+          and targets.shape == (logits.shape[0],), "targets: contiguous CUDA int64 [B]")
+    _need(reduction in GH_REDUCTION, "reduction must be 'mean' or 'sum'")
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=logits.device)
+    _need(loss.dtype == torch.float32 and loss.numel() == 1, "loss must be a float32 scalar")
+    if row_loss is not None:
+        _need(row_loss.dtype == torch.float32 and row_loss.is_cuda and row_loss.is_contiguous()
+              and row_loss.shape == (logits.shape[0],), "row_loss: contiguous CUDA float32 [B]")
+    B, V = logits.shape
+    dtype = GH_F32 if logits.dtype == torch.float32 else GH_BF16
+    st = lib().gh_ce_fwd(_ptr(logits), _ptr(targets), B, V, dtype, int(ignore_index), GH_REDUCTION[reduction],
+                         float(z_loss), _ptr(loss), _ptr(row_loss), _stream_handle(stream))
+    _check(st, "gh_ce_fwd")
+    return loss, row_loss
+
+
+def gh_selective_log_softmax(logits, index, *, out=None, stream=None):
+    """``log_softmax(logits)[..., index]`` per row without the full log-probabilities
+    (one call into ``gh_selective_log_softmax``).
+
+    ``logits`` CUDA [..., V] float32 or bfloat16, contiguous; ``index`` CUDA
+    int64 [...] (the leading shape of ``logits``).  Returns float32 [...]; an
+    index outside [0, V) gives NaN in its row and sets GH_ERR_TARGET_RANGE in
+    the device status.
+    """
+    import torch
+    _need(logits.dim() >= 1 and logits.is_cuda and logits.is_contiguous(), "logits: contiguous CUDA [..., V]")
+    _need(logits.dtype in (torch.float32, torch.bfloat16), "logits dtype must be float32 or bfloat16")
+    _need(index.dtype == torch.int64 and index.is_cuda and index.is_contiguous()
+          and tuple(index.shape) == tuple(logits.shape[:-1]), "index: contiguous CUDA int64 [...]")
+    if out is None:
+        out = torch.empty(index.shape, dtype=torch.float32, device=logits.device)
+    _need(out.dtype == torch.float32 and out.is_contiguous() and tuple(out.shape) == tuple(index.shape),
+          "out: contiguous float32 [...]")
+    V = logits.shape[-1]
+    rows = index.numel()
+    dtype = GH_F32 if logits.dtype == torch.float32 else GH_BF16
+    st = lib().gh_selective_log_softmax(_ptr(logits), _ptr(index), rows, V, dtype, _ptr(out),
+                                        _stream_handle(stream))
+    _check(st, "gh_selective_log_softmax")
+    return out
 
 
 def gh_linear_ce(inputs, weight, targets, ignore_index: int = -100, reduction: str = "mean",

@@ -121,6 +121,73 @@ gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B,
   return st;
 }
 
+gh_status_t gh_ce_fwd(const void* logits, const int64_t* targets, int64_t B, int64_t V, gh_dtype_t dtype,
+                     int64_t ignore_index, gh_reduction_t reduction, float z_mult, float* loss, float* row_loss_out,
+                     void* stream_) {
+  if (B < 0 || V < 1 || V >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
+  if (dtype != GH_F32 && dtype != GH_BF16) return GH_ERR_INVALID_ARG;
+  if (reduction != GH_REDUCTION_MEAN && reduction != GH_REDUCTION_SUM) return GH_ERR_INVALID_ARG;
+  if (!std::isfinite(z_mult)) return GH_ERR_INVALID_ARG;
+  if (!loss) return GH_ERR_INVALID_ARG;
+  if (B > 0 && (!logits || !targets)) return GH_ERR_INVALID_ARG;
+  const int es = dtype == GH_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(logits) % es) || (reinterpret_cast<uintptr_t>(targets) % 8) ||
+      (reinterpret_cast<uintptr_t>(loss) % 4) || (reinterpret_cast<uintptr_t>(row_loss_out) % 4))
+    return GH_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (B == 0) return cudaMemsetAsync(loss, 0, sizeof(float), stream) == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+
+  // Scratch: the valid-target count, and the row losses unless the caller
+  // takes them.
+  void* scratch = nullptr;
+  const size_t rows_bytes = row_loss_out ? 0 : static_cast<size_t>(B) * sizeof(float);
+  gh_status_t st = scratch_alloc(&scratch, 16 + rows_bytes, stream);
+  if (st != GH_OK) return st;
+  unsigned long long* n_valid = static_cast<unsigned long long*>(scratch);
+  float* row_loss = row_loss_out ? row_loss_out : reinterpret_cast<float*>(static_cast<char*>(scratch) + 16);
+
+  const int mean = reduction == GH_REDUCTION_MEAN;
+  st = ce_count_launch(targets, B, V, ignore_index, n_valid, stream);
+  if (st == GH_OK) {
+    CeArgs a{};
+    a.logits = logits;
+    a.targets = targets;
+    a.V = V;
+    a.ld = V;
+    a.ignore_index = ignore_index;
+    a.z = z_mult;
+    a.mean = mean;
+    a.row_loss = row_loss;
+    a.mode = kModeFwd;
+    st = ce_launch(a, B, dtype, stream);
+  }
+  if (st == GH_OK) st = ce_reduce_launch(row_loss, B, n_valid, mean, loss, stream);
+  scratch_free(scratch, stream);
+  return st;
+}
+
+gh_status_t gh_selective_log_softmax(const void* logits, const int64_t* index, int64_t rows, int64_t V,
+                                     gh_dtype_t dtype, float* out, void* stream_) {
+  if (rows < 0 || V < 1 || V >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
+  if (dtype != GH_F32 && dtype != GH_BF16) return GH_ERR_INVALID_ARG;
+  if (rows > 0 && (!logits || !index || !out)) return GH_ERR_INVALID_ARG;
+  const int es = dtype == GH_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(logits) % es) || (reinterpret_cast<uintptr_t>(index) % 8) ||
+      (reinterpret_cast<uintptr_t>(out) % 4))
+    return GH_ERR_INVALID_ARG;
+  if (rows == 0) return GH_OK;
+  CeArgs a{};
+  a.logits = logits;
+  a.targets = index;
+  a.V = V;
+  a.ld = V;
+  a.ignore_index = INT64_MIN;  // every in-range index is selected
+  a.row_loss = out;
+  a.mode = kModeSelect;
+  a.profile_kind = GH_KERNEL_CE_ROW;
+  return ce_launch(a, rows, dtype, static_cast<cudaStream_t>(stream_));
+}
+
 gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* targets, int64_t N, int64_t D,
                          int64_t V, int64_t chunk, gh_accum_t accum_dtype, int64_t ignore_index,
                          gh_reduction_t reduction, float z_mult, float* loss, void* grad_inputs, void* grad_weight,

@@ -22,11 +22,13 @@
 #include <climits>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include <cuda_fp16.h>
 
 #include "ce.h"
+#include "ce_device.cuh"
 #include "common.cuh"
 #include "profile.h"
 
@@ -34,197 +36,6 @@ namespace gh {
 
 namespace {
 
-template <typename T>
-struct Elem;
-template <>
-struct Elem<float> {
-  static constexpr int kBytes = 4;
-  static __device__ __forceinline__ float load(const void* p) { return *reinterpret_cast<const float*>(p); }
-  static __device__ __forceinline__ void store(void* p, float v) { *reinterpret_cast<float*>(p) = v; }
-};
-template <>
-struct Elem<uint16_t> {  // bf16 bit pattern
-  static constexpr int kBytes = 2;
-  static __device__ __forceinline__ float load(const void* p) {
-    return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p)) << 16);
-  }
-  static __device__ __forceinline__ void store(void* p, float v) {
-    *reinterpret_cast<uint16_t*>(p) = to_bf16_bits(v);
-  }
-};
-
-constexpr float kNegInf = -__builtin_huge_valf();
-
-template <typename T>
-__device__ __forceinline__ T neg_inf_elem();
-template <>
-__device__ __forceinline__ float neg_inf_elem<float>() { return kNegInf; }
-template <>
-__device__ __forceinline__ uint16_t neg_inf_elem<uint16_t>() { return 0xff80u; }
-
-// Unpack one 16-byte chunk into floats.
-template <typename T>
-__device__ __forceinline__ void unpack16(const uint4& q, float (&v)[16 / Elem<T>::kBytes]);
-template <>
-__device__ __forceinline__ void unpack16<float>(const uint4& q, float (&v)[4]) {
-  v[0] = __uint_as_float(q.x);
-  v[1] = __uint_as_float(q.y);
-  v[2] = __uint_as_float(q.z);
-  v[3] = __uint_as_float(q.w);
-}
-template <>
-__device__ __forceinline__ void unpack16<uint16_t>(const uint4& q, float (&v)[8]) {
-  v[0] = bf16_lo(q.x); v[1] = bf16_hi(q.x);
-  v[2] = bf16_lo(q.y); v[3] = bf16_hi(q.y);
-  v[4] = bf16_lo(q.z); v[5] = bf16_hi(q.z);
-  v[6] = bf16_lo(q.w); v[7] = bf16_hi(q.w);
-}
-
-template <typename T>
-__device__ __forceinline__ uint4 pack16(const float (&g)[16 / Elem<T>::kBytes]);
-template <>
-__device__ __forceinline__ uint4 pack16<float>(const float (&g)[4]) {
-  return make_uint4(__float_as_uint(g[0]), __float_as_uint(g[1]), __float_as_uint(g[2]), __float_as_uint(g[3]));
-}
-template <>
-__device__ __forceinline__ uint4 pack16<uint16_t>(const float (&g)[8]) {
-  return make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]), pack_bf16x2(g[4], g[5]),
-                    pack_bf16x2(g[6], g[7]));
-}
-
-// Online (max, sum of exp(x - max)) state.  Combining is exact up to rounding
-// and never forms (-inf) - (-inf).
-struct MaxSum {
-  float m, s;
-};
-
-__device__ __forceinline__ MaxSum combine(MaxSum a, MaxSum b) {
-  const float M = fmaxf(a.m, b.m);
-  if (M == kNegInf) return {kNegInf, 0.0f};
-  const float sa = (a.m == kNegInf) ? 0.0f : a.s * ex2((a.m - M) * kLog2e);
-  const float sb = (b.m == kNegInf) ? 0.0f : b.s * ex2((b.m - M) * kLog2e);
-  return {M, sa + sb};
-}
-
-// Fold the 16/ES values of one chunk into the running state.
-template <int N>
-__device__ __forceinline__ void fold_chunk(MaxSum& st, const float (&v)[N]) {
-  float cm = v[0];
-#pragma unroll
-  for (int i = 1; i < N; ++i) cm = fmaxf(cm, v[i]);
-  if (cm == kNegInf) return;  // chunk of padding / -inf logits only
-  if (cm > st.m) {
-    st.s = (st.m == kNegInf) ? 0.0f : st.s * ex2((st.m - cm) * kLog2e);
-    st.m = cm;
-  }
-  const float nm = -st.m * kLog2e;
-  float acc = 0.0f;
-#pragma unroll
-  for (int i = 0; i < N; ++i) acc += ex2(fmaf(v[i], kLog2e, nm));
-  st.s += acc;
-}
-
-__device__ __forceinline__ MaxSum warp_reduce(MaxSum st) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    MaxSum other{__shfl_xor_sync(0xffffffffu, st.m, o), __shfl_xor_sync(0xffffffffu, st.s, o)};
-    st = combine(st, other);
-  }
-  return st;
-}
-
-// Block-wide reduction in a fixed order; every thread gets the result.
-template <int kThreads>
-__device__ __forceinline__ MaxSum block_reduce(MaxSum st, float* scratch /* 2*kWarps */) {
-  constexpr int kWarps = kThreads / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  st = warp_reduce(st);
-  if (lane == 0) {
-    scratch[2 * warp] = st.m;
-    scratch[2 * warp + 1] = st.s;
-  }
-  __syncthreads();
-  MaxSum r{kNegInf, 0.0f};
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) r = combine(r, MaxSum{scratch[2 * w], scratch[2 * w + 1]});
-  __syncthreads();
-  return r;
-}
-
-// Block-wide max / sum; every thread gets the result.  `scratch` holds one
-// float per warp and is not reused, so one barrier suffices.
-template <int kThreads>
-__device__ __forceinline__ float block_max(float v, float* scratch) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = scratch[0];
-#pragma unroll
-  for (int w = 1; w < kThreads / 32; ++w) r = fmaxf(r, scratch[w]);
-  return r;
-}
-
-template <int kThreads>
-__device__ __forceinline__ float block_sum(float v, float* scratch) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = scratch[0];
-#pragma unroll
-  for (int w = 1; w < kThreads / 32; ++w) r += scratch[w];
-  return r;
-}
-
-template <int N>
-__device__ __forceinline__ float tree_sum(const float (&e)[N]) {
-  if constexpr (N == 8) {
-    return ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-  } else {
-    return (e[0] + e[1]) + (e[2] + e[3]);
-  }
-}
-
-__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ uint4 pack_f16x8(const float (&e)[8]) {
-  return make_uint4(pack_f16x2(e[0], e[1]), pack_f16x2(e[2], e[3]), pack_f16x2(e[4], e[5]),
-                    pack_f16x2(e[6], e[7]));
-}
-template <int N>
-__device__ __forceinline__ uint4 pack_f16x8(const float (&e)[N]) {  // fp32 rows keep their values
-  return make_uint4(0, 0, 0, 0);
-}
-
-__device__ __forceinline__ float2 f16x2_to_f32(uint32_t w) {
-  __half2 h;
-  memcpy(&h, &w, sizeof(h));
-  return __half22float2(h);
-}
-
-__device__ __forceinline__ float f16_to_f32(uint16_t h) {
-  float f;
-  asm("{\n\t.reg .f16 x;\n\tmov.b16 x, %1;\n\tcvt.f32.f16 %0, x;\n\t}" : "=f"(f) : "h"(h));
-  return f;
-}
-
-template <int N>
-__device__ __forceinline__ void unpack_f16x8(const uint4& q, float (&g)[N]) {
-  const float2 a = f16x2_to_f32(q.x), b = f16x2_to_f32(q.y), c = f16x2_to_f32(q.z), d = f16x2_to_f32(q.w);
-  g[0] = a.x; g[1] = a.y; g[2] = b.x; g[3] = b.y;
-  if constexpr (N == 8) { g[4] = c.x; g[5] = c.y; g[6] = d.x; g[7] = d.y; }
-}
 
 #ifndef GH_CE_ROW_THREADS
 #define GH_CE_ROW_THREADS 512
@@ -381,7 +192,7 @@ __global__ void __launch_bounds__(1024) ce_count1_kernel(const int64_t* __restri
 //      owner afterwards with the -scale term.
 // fp32 rows only sum in pass 1 and re-evaluate the exponent in pass 2 (a
 // cache would not fit in place).
-template <typename T>
+template <typename T, int MODE>
 __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
   constexpr int NG = 2;                 // row groups per CTA
   constexpr int ES = Elem<T>::kBytes;
@@ -432,7 +243,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
   uint32_t valid_rows = 0;  // selects the exchange barrier and record buffer
   uint32_t xphase = 0;      // bit pb: parity of the next wait on xbar[grp][pb]
   bool ok = true;
-  const unsigned long long nv = *a.n_valid;
+  constexpr bool with_grad = MODE == kModeFwdBwd;
+  const unsigned long long nv = with_grad ? *a.n_valid : 1ull;
   const float scale = a.mean ? 1.0f / static_cast<float>(nv > 0 ? nv : 1ull) : 1.0f;
 
   for (int64_t k = 0; row_of(k) < a.B; ++k) {
@@ -445,8 +257,17 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
     const SliceGeo g = slice_geo<ES>(a, row, rank);
 
     if (!target_valid(a, t)) {
-      // Ignored row: zero gradient, zero loss, the logits are never read.
-      if (rank == 0 && leader) a.row_loss[row] = 0.0f;
+      // Ignored row: zero gradient, zero loss, the logits are never read.  An
+      // out-of-range index of the selective log-softmax gives NaN.
+      if (rank == 0 && leader) {
+        if constexpr (MODE == kModeSelect) {
+          a.row_loss[row] = __int_as_float(0x7fc00000);
+          record_status(GH_ERR_TARGET_RANGE);
+        } else {
+          a.row_loss[row] = 0.0f;
+        }
+      }
+      if constexpr (with_grad) {
       const int glead = static_cast<int>(reinterpret_cast<uintptr_t>(g.gdst) & 15);
       const int gspan = glead + g.n * ES;
       const int z_lo = (glead + 15) >> 4, z_hi = max(z_lo, gspan >> 4);
@@ -456,6 +277,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
       const int kt = max(h, (16 * z_hi - glead) / ES);
       for (int e = tid; e < h; e += NT) Elem<T>::store(g.gdst + e * ES, 0.0f);
       for (int e = kt + tid; e < g.n; e += NT) Elem<T>::store(g.gdst + e * ES, 0.0f);
+      }
     } else {
       // ---- pass 0: this thread's max, piece by piece as copies land ----------------------
       const int nb = g.x_hi - g.x_lo;
@@ -557,14 +379,14 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
           for (int u = 0; u < kUnroll; ++u) {
             float e[EPC];
             exps(q[u], e);
-            if constexpr (kBf16) *reinterpret_cast<uint4*>(buf + 16 * (c + u * NT)) = pack_f16x8(e);
+            if (kBf16 && with_grad) *reinterpret_cast<uint4*>(buf + 16 * (c + u * NT)) = pack_f16x8(e);
           }
         }
         for (; c < g.nchunks; c += NT) {
           uint4* p0 = reinterpret_cast<uint4*>(buf + 16 * c);
           float e0[EPC];
           exps(*p0, e0);
-          if constexpr (kBf16) *p0 = pack_f16x8(e0);
+          if (kBf16 && with_grad) *p0 = pack_f16x8(e0);
         }
         s_t = acc.x + acc.y;
       }
@@ -623,7 +445,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
       gsync();
       const float lse = sh.lse[grp];
       ++valid_rows;
-      if (rank == 0 && leader) a.row_loss[row] = (lse - sh.xt[grp]) + a.z * lse * lse;
+      if (rank == 0 && leader)
+        a.row_loss[row] = MODE == kModeSelect ? sh.xt[grp] - lse : (lse - sh.xt[grp]) + a.z * lse * lse;
 
       // ---- pass 2: gradient straight to global -------------------------------------------
       const float coef = scale * (1.0f + 2.0f * a.z * lse);
@@ -654,7 +477,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
           if (16 * c + j * ES >= g.lead && e < g.n) Elem<T>::store(g.gdst + e * ES, gv[j]);
         }
       };
-      if (ok) {
+      if (ok && with_grad) {
         if (a.congruent) {
           uint8_t* dbase = g.gdst - g.lead;
           int c = g.c_lo + ((tid - g.c_lo) % NT + NT) % NT;
@@ -718,7 +541,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) ce_row_kernel(CeArgs a) {
 
 // Rows too long for the shared-memory path: one CTA per row, two passes over
 // global memory.  Element loads/stores are scalar at the row's unaligned ends.
-template <typename T>
+template <typename T, int MODE>
 __global__ void __launch_bounds__(kStreamThreads) ce_stream_kernel(CeArgs a) {
   constexpr int ES = Elem<T>::kBytes;
   constexpr int EPC = 16 / ES;
@@ -740,9 +563,18 @@ __global__ void __launch_bounds__(kStreamThreads) ce_stream_kernel(CeArgs a) {
   const int64_t kt = tmax<int64_t>(h, (16 * c_hi - lead) / ES);
   const uint8_t* sbase = src - lead;
 
+  constexpr bool with_grad = MODE == kModeFwdBwd;
   if (!valid) {
-    if (tid == 0) a.row_loss[row] = 0.0f;
-    for (int64_t k = tid; k < V; k += kStreamThreads) Elem<T>::store(dst + k * ES, 0.0f);
+    if (tid == 0) {
+      if constexpr (MODE == kModeSelect) {
+        a.row_loss[row] = __int_as_float(0x7fc00000);
+        record_status(GH_ERR_TARGET_RANGE);
+      } else {
+        a.row_loss[row] = 0.0f;
+      }
+    }
+    if (with_grad)
+      for (int64_t k = tid; k < V; k += kStreamThreads) Elem<T>::store(dst + k * ES, 0.0f);
     return;
   }
   MaxSum st{kNegInf, 0.0f};
@@ -763,7 +595,8 @@ __global__ void __launch_bounds__(kStreamThreads) ce_stream_kernel(CeArgs a) {
   st = block_reduce<kStreamThreads>(st, red);
   const float lse = st.m + logf(st.s);
   const float xt = Elem<T>::load(src + t * ES);
-  if (tid == 0) a.row_loss[row] = (lse - xt) + a.z * lse * lse;
+  if (tid == 0) a.row_loss[row] = MODE == kModeSelect ? xt - lse : (lse - xt) + a.z * lse * lse;
+  if constexpr (!with_grad) return;
 
   const unsigned long long nv = *a.n_valid;
   const float scale = a.mean ? 1.0f / static_cast<float>(nv > 0 ? nv : 1ull) : 1.0f;
@@ -868,7 +701,23 @@ static int device_sm_count() {
 
 namespace {
 
-void (*row_kernel_for(int es))(CeArgs) { return es == 4 ? ce_row_kernel<float> : ce_row_kernel<uint16_t>; }
+using CeKernel = void (*)(CeArgs);
+
+template <typename T>
+CeKernel row_kernel_mode(int mode) {
+  return mode == kModeSelect ? ce_row_kernel<T, kModeSelect>
+         : mode == kModeFwd  ? ce_row_kernel<T, kModeFwd>
+                             : ce_row_kernel<T, kModeFwdBwd>;
+}
+CeKernel row_kernel_for(int es, int mode) {
+  return es == 4 ? row_kernel_mode<float>(mode) : row_kernel_mode<uint16_t>(mode);
+}
+template <typename T>
+CeKernel stream_kernel_mode(int mode) {
+  return mode == kModeSelect ? ce_stream_kernel<T, kModeSelect>
+         : mode == kModeFwd  ? ce_stream_kernel<T, kModeFwd>
+                             : ce_stream_kernel<T, kModeFwdBwd>;
+}
 
 // Launch plan of the row kernel for one (device, V, element size), computed
 // once: the occupancy queries and attribute calls cost far more than a launch.
@@ -898,16 +747,19 @@ gh_status_t row_plan(int64_t V, int es, CePlan* out, int64_t* active_out) {
   CePlan plan = ce_plan(V, es);
   int64_t active = 0;
   if (!plan.streaming) {
-    void (*kern)(CeArgs) = row_kernel_for(es);
+    CeKernel kern = row_kernel_for(es, kModeFwdBwd);
     // The dynamic shared memory limit is an attribute of the kernel, shared by
-    // every plan: raise it once per device to the opt-in maximum.
+    // every plan: raise it once per device to the opt-in maximum, for the
+    // kernel of every mode (they share one launch plan).
     static bool raised[64][2] = {};
     const int kv = es == 4;
     if (dev < 64 && !raised[dev][kv]) {
       int optin = 0;
       if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return GH_ERR_CUDA;
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess)
-        return GH_ERR_CUDA;
+      for (int m : {kModeFwdBwd, kModeFwd, kModeSelect})
+        if (cudaFuncSetAttribute(row_kernel_for(es, m), cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
+            cudaSuccess)
+          return GH_ERR_CUDA;
       raised[dev][kv] = true;
     }
     // Clusters must fit inside a GPC, so the number resident at once depends on
@@ -948,10 +800,28 @@ gh_status_t row_plan(int64_t V, int es, CePlan* out, int64_t* active_out) {
 
 }  // namespace
 
+// Forward-only rows take the ring pipeline (ce_fwd.cu) when there are enough
+// rows to keep every SM's ring busy (round-robin rows: at least kRingMinRowsPerSm
+// per SM keeps the last wave's imbalance small); fewer rows take the row
+// kernel, whose clusters split long rows over several SMs.  GH_CE_FWD_PATH=ring
+// or =rows forces one of the two (tests).
+constexpr int kRingMinRowsPerSm = 8;
+
+static bool use_ring(int64_t B, int sms) {
+  const char* e = std::getenv("GH_CE_FWD_PATH");
+  if (e && std::strcmp(e, "ring") == 0) return true;
+  if (e && std::strcmp(e, "rows") == 0) return false;
+  return B >= static_cast<int64_t>(kRingMinRowsPerSm) * sms;
+}
+
 gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaStream_t stream) {
   CeArgs a = args_in;
   a.B = B;
   const int es = dtype == GH_F32 ? 4 : 2;
+  if (a.mode != kModeFwdBwd) {
+    const int sms = device_sm_count();
+    if (use_ring(B, sms)) return ce_ring_launch(a, es, static_cast<int>(std::min<int64_t>(B, sms)), stream);
+  }
   CePlan plan;
   int64_t active = 0;
   gh_status_t st = row_plan(a.V, es, &plan, &active);
@@ -964,16 +834,13 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
   if (plan.streaming) {
     if (B > INT32_MAX) return GH_ERR_UNSUPPORTED;
     ProfileScope prof(a.profile_kind, stream);
-    const cudaError_t e = dtype == GH_F32
-                              ? launch_pdl(ce_stream_kernel<float>, dim3(static_cast<unsigned>(B)), dim3(kStreamThreads),
-                                           0, stream, 1, a)
-                              : launch_pdl(ce_stream_kernel<uint16_t>, dim3(static_cast<unsigned>(B)),
-                                           dim3(kStreamThreads), 0, stream, 1, a);
+    const CeKernel sk = es == 4 ? stream_kernel_mode<float>(a.mode) : stream_kernel_mode<uint16_t>(a.mode);
+    const cudaError_t e = launch_pdl(sk, dim3(static_cast<unsigned>(B)), dim3(kStreamThreads), 0, stream, 1, a);
     note_launch();
     return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
   }
 
-  void (*kern)(CeArgs) = row_kernel_for(es);
+  const CeKernel kern = row_kernel_for(es, a.mode);
   // Persistent grid: as many clusters as can be resident at once, no more
   // than there are rows (two per cluster, one per row group).
   const int64_t nclusters = std::min<int64_t>(active, (B + 1) / 2);

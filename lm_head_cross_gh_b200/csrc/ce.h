@@ -8,6 +8,13 @@
 
 namespace gh {
 
+// What the row kernel produces per row.
+enum CeMode : int {
+  kModeFwdBwd = 0,   // row loss and the logits gradient
+  kModeFwd = 1,      // row loss only (no gradient; grad may be null)
+  kModeSelect = 2    // row value x[index] - lse (selective log-softmax; NaN for an index outside [0, V))
+};
+
 struct CeArgs {
   const void* logits;                 // [B, V] row-major
   void* grad;                         // [B, V] row-major, same dtype
@@ -18,7 +25,7 @@ struct CeArgs {
   float z;                            // z-loss multiplier
   int mean;                           // 1: divide by n_valid
   const unsigned long long* n_valid;  // written by ce_count_kernel
-  float* row_loss;                    // [B] scratch
+  float* row_loss;                    // [B] per-row values (losses, or the selected log-probabilities)
   int64_t B;                          // rows (set by ce_launch)
   int slice;                          // elements per CTA (set by ce_launch)
   int cluster;                        // CTAs per row (set by ce_launch)
@@ -26,6 +33,7 @@ struct CeArgs {
   int npieces;                        // bulk copies per slice (set by ce_launch)
   int congruent;                      // (logits - grad) % 16 == 0
   int profile_kind;                   // gh_kernel_t the row kernel is timed as
+  int mode;                           // CeMode
 };
 
 struct CePlan {
@@ -40,6 +48,10 @@ CePlan ce_plan(int64_t V, int elem_bytes);
 gh_status_t ce_count_launch(const int64_t* targets, int64_t n, int64_t V, int64_t ii,
                             unsigned long long* count, cudaStream_t stream);
 gh_status_t ce_launch(const CeArgs& args, int64_t B, gh_dtype_t dtype, cudaStream_t stream);
+// Forward-only ring pipeline (ce_fwd.cu): modes kModeFwd and kModeSelect,
+// one persistent CTA per SM (`grid` CTAs), rows round-robin over the CTAs.
+int ce_ring_smem_bytes();
+gh_status_t ce_ring_launch(const CeArgs& args, int elem_bytes, int grid, cudaStream_t stream);
 gh_status_t ce_reduce_launch(const float* row_loss, int64_t B, const unsigned long long* n_valid, int mean,
                              float* loss, cudaStream_t stream);
 

@@ -1,0 +1,402 @@
+// Forward-only cross-entropy rows (the loss without its gradient, and the
+// selective log-softmax x[index] - lse) as one streaming pipeline per SM.
+//
+// Without a gradient pass nothing has to stay in shared memory once it has
+// been read, so the row-buffer design of the forward+backward kernel (a whole
+// row resident, the next row's copy waiting for the buffer) gives way to a ring
+// of fixed-size pieces that runs across row boundaries:
+//
+//   warp 16 (producer)   walks this CTA's rows and their pieces in order and
+//                        starts a bulk copy into the next free ring slot;
+//   warps 0-15 (consumers, four groups of four warps)
+//                        piece n goes whole to group n % 4: as it lands, each
+//                        thread loads its eight chunks into registers, the
+//                        group frees the slot at once, and the thread folds the
+//                        chunks into its online (max, sum of exp) state;
+//                        at a row's end each warp reduces its state and posts
+//                        it to the row's finalizer;
+//   warps 17-20 (finalizers)
+//                        take the valid rows in turn (row k to warp 17 + k % 4);
+//                        each merges the 16 warp states with the row's ragged
+//                        ends (the elements outside the whole 16-byte chunks,
+//                        read from global), reads the target logit and writes
+//                        the row value.  With four of them, a finalizer's
+//                        global loads for a row have about four rows' time
+//                        to arrive before the row's states do.
+//
+// Every logit is read from HBM once and every element costs one exponential;
+// the consumers never wait on each other, and the producer stays up to
+// kRingSlots pieces (192 KiB) ahead.  Rows are assigned round-robin to the
+// persistent CTAs; all barriers are mbarriers with bounded waits.
+#include "ce.h"
+#include "ce_device.cuh"
+#include "common.cuh"
+#include "profile.h"
+
+namespace gh {
+
+namespace {
+
+constexpr int kRingConsumerWarps = 16;
+constexpr int kRingConsumers = 32 * kRingConsumerWarps;
+// The consumers form kRingGroups groups; piece n goes to group n % kRingGroups
+// whole, so each group's warps (one per SM sub-partition) run out of phase
+// with the other groups' and one group's loads and max overlap another's
+// exponentials.
+constexpr int kRingGroups = 4;
+constexpr int kGroupWarps = kRingConsumerWarps / kRingGroups;
+constexpr int kGroupThreads = 32 * kGroupWarps;
+constexpr int kRingFinalizers = 4;                 // warps; also the row-state buffers in flight
+constexpr int kRingThreads = kRingConsumers + 32 + 32 * kRingFinalizers;  // + producer warp
+constexpr int kRingSlots = 12;
+constexpr int kRingPieceBytes = 16384;
+constexpr int kRingPieceChunks = kRingPieceBytes / 16;
+constexpr int kPieceChunksPerThread = kRingPieceChunks / kGroupThreads;  // 8
+static_assert(kRingSlots % kRingGroups == 0, "a slot always serves the same group");
+static_assert(kRingPieceChunks % kGroupThreads == 0, "whole chunks per thread");
+constexpr int kRingHdrBytes = 1024;
+
+struct RingShared {
+  uint64_t full[kRingSlots];   // piece landed (producer's expect_tx + the copy's bytes)
+  uint64_t empty[kRingSlots];  // piece consumed (one arrival per warp of its group)
+  uint64_t rowfull[kRingFinalizers];   // per valid row k % 4: every consumer warp posted its state
+  uint64_t rowempty[kRingFinalizers];  // per valid row k % 4: its finalizer has read the states
+  float2 part[kRingFinalizers][kRingConsumerWarps];
+  int abort;                   // a wait ran out: every role stops waiting
+};
+static_assert(sizeof(RingShared) <= kRingHdrBytes, "ring header too large");
+
+// Byte geometry of one row: chunks [c_lo, c_hi) (16-byte, counted from the
+// row's first byte rounded down to 16) lie wholly inside the row and are
+// copied in bulk; the h head elements [0, h) and the tail elements [tail, V)
+// are the ragged ends, read element by element.
+struct RingRow {
+  const uint8_t* base;  // row start rounded down to 16 bytes
+  int c_lo, c_hi, h, tail;
+};
+
+template <int ES>
+__device__ __forceinline__ RingRow ring_row(const CeArgs& a, int64_t row) {
+  RingRow r;
+  const uint8_t* src = static_cast<const uint8_t*>(a.logits) + row * a.ld * ES;
+  const int lead = static_cast<int>(reinterpret_cast<uintptr_t>(src) & 15);
+  const int64_t span = lead + a.V * ES;
+  r.base = src - lead;
+  r.c_lo = (lead + 15) >> 4;
+  r.c_hi = static_cast<int>(tmax<int64_t>(r.c_lo, span >> 4));
+  r.h = static_cast<int>(tmin<int64_t>(a.V, (16 * r.c_lo - lead) / ES));
+  r.tail = static_cast<int>(tmax<int64_t>(r.h, (16 * static_cast<int64_t>(r.c_hi) - lead) / ES));
+  return r;
+}
+
+__device__ __forceinline__ int ring_pieces(const RingRow& r) {
+  return (r.c_hi - r.c_lo + kRingPieceChunks - 1) / kRingPieceChunks;
+}
+
+__device__ __forceinline__ bool ring_target_valid(const CeArgs& a, int64_t t) {
+  return (t != a.ignore_index) && t >= 0 && t < a.V;
+}
+
+// The running reference of a thread's online sum is its max so far plus
+// kRingBump: a rescale happens only when a chunk beats the reference, so a row
+// whose values keep creeping upwards rescales once per kRingBump of growth
+// instead of once per chunk (each rescale costs an approximate exponential's
+// rounding).  Terms then sit at or below exp(-kRingBump); fp32 keeps every term
+// within ~79 of the max, and the rest are below 1e-34 of the sum.
+constexpr float kRingBump = 8.0f;
+
+__device__ __forceinline__ void raise_ref(MaxSum& st, float cm) {
+  if (cm > st.m) {
+    const float mn = cm + kRingBump;
+    st.s = (st.m == kNegInf) ? 0.0f : st.s * ex2((st.m - mn) * kLog2e);
+    st.m = mn;
+  }
+}
+
+// One thread's share of a full piece: chunks gtid + i * kGroupThreads
+// (i < 8), already in registers.  One max test and at most one rescale cover
+// all eight, and the exponentials go to four independent accumulators.
+template <typename T>
+__device__ __forceinline__ void fold_full_piece(MaxSum& st, const uint4 (&q)[kPieceChunksPerThread]) {
+  constexpr int EPC = 16 / Elem<T>::kBytes;
+  constexpr int K = kPieceChunksPerThread;
+  float cm;
+  if constexpr (EPC == 8) {
+    uint32_t m4[4] = {q[0].x, q[0].y, q[0].z, q[0].w};
+#pragma unroll
+    for (int i = 1; i < K; ++i) {
+      m4[0] = bf16x2_max(m4[0], q[i].x);
+      m4[1] = bf16x2_max(m4[1], q[i].y);
+      m4[2] = bf16x2_max(m4[2], q[i].z);
+      m4[3] = bf16x2_max(m4[3], q[i].w);
+    }
+    const uint32_t mx = bf16x2_max(bf16x2_max(m4[0], m4[1]), bf16x2_max(m4[2], m4[3]));
+    cm = fmaxf(bf16_lo(mx), bf16_hi(mx));
+  } else {
+    float m4[4] = {__uint_as_float(q[0].x), __uint_as_float(q[0].y), __uint_as_float(q[0].z),
+                   __uint_as_float(q[0].w)};
+#pragma unroll
+    for (int i = 1; i < K; ++i) {
+      m4[0] = fmaxf(m4[0], __uint_as_float(q[i].x));
+      m4[1] = fmaxf(m4[1], __uint_as_float(q[i].y));
+      m4[2] = fmaxf(m4[2], __uint_as_float(q[i].z));
+      m4[3] = fmaxf(m4[3], __uint_as_float(q[i].w));
+    }
+    cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+  }
+  raise_ref(st, cm);
+  if (st.m == kNegInf) return;  // only -inf logits so far
+  const float nm = -st.m * kLog2e;
+  const float2 l2 = make_float2(kLog2e, kLog2e), nm2 = make_float2(nm, nm);
+  float2 acc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                   make_float2(0.0f, 0.0f)};
+#pragma unroll
+  for (int i = 0; i < K; ++i) {
+    float v[EPC];
+    unpack16<T>(q[i], v);
+#pragma unroll
+    for (int j = 0; j < EPC; j += 2) {
+      const float2 y = __ffma2_rn(make_float2(v[j], v[j + 1]), l2, nm2);
+      float2& ac = acc[(i * EPC / 2 + j / 2) & 3];
+      ac = __fadd2_rn(ac, make_float2(ex2(y.x), ex2(y.y)));
+    }
+  }
+  const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 a = __fadd2_rn(a01, a23);
+  st.s += a.x + a.y;
+}
+
+// One chunk of a short piece (a row's last), folded on its own.
+template <typename T>
+__device__ __forceinline__ void fold_one(MaxSum& st, const uint4& q) {
+  constexpr int EPC = 16 / Elem<T>::kBytes;
+  float v[EPC];
+  unpack16<T>(q, v);
+  float cm = v[0];
+#pragma unroll
+  for (int i = 1; i < EPC; ++i) cm = fmaxf(cm, v[i]);
+  raise_ref(st, cm);
+  if (st.m == kNegInf) return;
+  const float nm = -st.m * kLog2e;
+  float acc = 0.0f;
+#pragma unroll
+  for (int i = 0; i < EPC; ++i) acc += ex2(fmaf(v[i], kLog2e, nm));
+  st.s += acc;
+}
+
+template <typename T, int MODE>
+__global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
+  constexpr int ES = Elem<T>::kBytes;
+  extern __shared__ __align__(128) uint8_t smem[];
+  RingShared& sh = *reinterpret_cast<RingShared*>(smem);
+  uint8_t* ring = smem + kRingHdrBytes;
+  const int warp = static_cast<int>(threadIdx.x) >> 5, lane = static_cast<int>(threadIdx.x) & 31;
+  const int64_t G = gridDim.x;
+  const int64_t first = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRingSlots; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.empty[i], kGroupWarps);
+    }
+    for (int i = 0; i < kRingFinalizers; ++i) {
+      mbar_init(&sh.rowfull[i], kRingConsumerWarps);
+      mbar_init(&sh.rowempty[i], 1);
+    }
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  pdl_wait();     // the predecessor's outputs (targets, logits) are complete
+  pdl_trigger();  // persistent grid: the next kernel may start launching
+  __syncthreads();
+
+  volatile int* abort_flag = &sh.abort;
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *abort_flag = 1;
+    return false;
+  };
+  auto target_of = [&](int64_t row) -> int64_t { return row < a.B ? a.targets[row] : int64_t(0); };
+
+  if (warp == kRingConsumerWarps) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      uint32_t n = 0;  // pieces issued
+      int64_t t = target_of(first);
+      for (int64_t row = first; row < a.B; row += G) {
+        const int64_t t_next = target_of(row + G);
+        if (ring_target_valid(a, t)) {
+          const RingRow r = ring_row<ES>(a, row);
+          const int np = ring_pieces(r);
+          for (int p = 0; p < np; ++p, ++n) {
+            const int s = static_cast<int>(n % kRingSlots);
+            if (!wait(&sh.empty[s], ((n / kRingSlots) & 1) ^ 1)) break;
+            const int c0 = r.c_lo + p * kRingPieceChunks;
+            const uint32_t bytes = 16u * static_cast<uint32_t>(tmin(kRingPieceChunks, r.c_hi - c0));
+            mbar_arrive_expect_tx(&sh.full[s], bytes);
+            bulk_g2s(ring + s * kRingPieceBytes, r.base + 16 * static_cast<int64_t>(c0), bytes, &sh.full[s]);
+          }
+        }
+        if (*abort_flag) break;
+        t = t_next;
+      }
+      // On an abort, the copies still in flight land before the CTA exits.
+      if (*abort_flag) {
+        for (uint32_t k = (n > kRingSlots ? n - kRingSlots : 0); k < n; ++k)
+          (void)mbar_wait(&sh.full[k % kRingSlots], (k / kRingSlots) & 1);
+      }
+    }
+    return;
+  }
+
+  if (warp > kRingConsumerWarps) {
+    // ---------------- finalizers ----------------
+    const uint32_t f = warp - kRingConsumerWarps - 1;
+    uint32_t k = 0;  // valid rows seen
+    uint32_t i = 0;  // rows seen
+    int64_t t = target_of(first);
+    for (int64_t row = first; row < a.B; row += G, ++i) {
+      const int64_t t_next = target_of(row + G);
+      if (!ring_target_valid(a, t)) {
+        if (lane == 0 && i % kRingFinalizers == f) {
+          if constexpr (MODE == kModeSelect) {
+            a.row_loss[row] = __int_as_float(0x7fc00000);
+            record_status(GH_ERR_TARGET_RANGE);
+          } else {
+            a.row_loss[row] = 0.0f;
+          }
+        }
+        t = t_next;
+        continue;
+      }
+      if (k % kRingFinalizers != f) {
+        ++k;
+        t = t_next;
+        continue;
+      }
+      const RingRow r = ring_row<ES>(a, row);
+      const uint8_t* src = static_cast<const uint8_t*>(a.logits) + row * a.ld * ES;
+      // ragged ends: lanes 0-15 the head elements, lanes 16-31 the tail
+      float edge = kNegInf;
+      if (lane < 16) {
+        if (lane < r.h) edge = Elem<T>::load(src + static_cast<int64_t>(lane) * ES);
+      } else {
+        const int64_t e = r.tail + (lane - 16);
+        if (e < a.V) edge = Elem<T>::load(src + e * ES);
+      }
+      const float xt = Elem<T>::load(src + t * ES);
+      const int j = static_cast<int>(f);
+      const bool ok = __all_sync(0xffffffffu, wait(&sh.rowfull[j], (k / kRingFinalizers) & 1));
+      MaxSum st = (lane < kRingConsumerWarps && ok) ? MaxSum{sh.part[j][lane].x, sh.part[j][lane].y}
+                                                    : MaxSum{kNegInf, 0.0f};
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.rowempty[j]);
+      st = combine(st, edge == kNegInf ? MaxSum{kNegInf, 0.0f} : MaxSum{edge, 1.0f});
+      st = warp_reduce(st);
+      if (lane == 0) {
+        const float lse = st.m + logf(st.s);
+        a.row_loss[row] = MODE == kModeSelect ? xt - lse : (lse - xt) + a.z * lse * lse;
+      }
+      ++k;
+      t = t_next;
+      if (!ok) break;
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int grp = warp / kGroupWarps;
+  const int gtid = static_cast<int>(threadIdx.x) - grp * kGroupThreads;
+  uint32_t n = 0;  // pieces seen (this group consumes n % kRingGroups == grp)
+  uint32_t k = 0;  // valid rows
+  int64_t t = target_of(first);
+  for (int64_t row = first; row < a.B; row += G) {
+    const int64_t t_next = target_of(row + G);
+    if (!ring_target_valid(a, t)) {
+      t = t_next;
+      continue;
+    }
+    const RingRow r = ring_row<ES>(a, row);
+    const int np = ring_pieces(r);
+    const int nbc = r.c_hi - r.c_lo;
+    MaxSum st{kNegInf, 0.0f};
+    bool ok = true;
+    for (int p = 0; p < np; ++p, ++n) {
+      if (static_cast<int>(n % kRingGroups) != grp) continue;
+      const int s = static_cast<int>(n % kRingSlots);
+      if (!__all_sync(0xffffffffu, wait(&sh.full[s], (n / kRingSlots) & 1))) {
+        ok = false;
+        break;
+      }
+      const uint8_t* piece = ring + s * kRingPieceBytes;
+      const int nc = tmin(kRingPieceChunks, nbc - p * kRingPieceChunks);
+      if (nc == kRingPieceChunks) {
+        // a full piece: into registers, the slot back to the producer (the
+        // arrive's release orders it after the loads), then the arithmetic
+        uint4 q[kPieceChunksPerThread];
+#pragma unroll
+        for (int i = 0; i < kPieceChunksPerThread; ++i)
+          q[i] = *reinterpret_cast<const uint4*>(piece + 16 * (gtid + i * kGroupThreads));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
+        fold_full_piece<T>(st, q);
+      } else {
+        for (int c = gtid; c < nc; c += kGroupThreads) fold_one<T>(st, *reinterpret_cast<const uint4*>(piece + 16 * c));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
+      }
+    }
+    if (!ok) break;
+    st = warp_reduce(st);
+    const int j = static_cast<int>(k % kRingFinalizers);
+    if (lane == 0) {
+      if (wait(&sh.rowempty[j], ((k / kRingFinalizers) & 1) ^ 1)) {
+        sh.part[j][warp] = make_float2(st.m, st.s);
+        mbar_arrive(&sh.rowfull[j]);
+      }
+    }
+    __syncwarp();
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+    ++k;
+    t = t_next;
+  }
+}
+
+using RingKernel = void (*)(CeArgs);
+
+template <typename T>
+RingKernel ring_kernel_mode(int mode) {
+  return mode == kModeSelect ? ce_ring_kernel<T, kModeSelect> : ce_ring_kernel<T, kModeFwd>;
+}
+
+RingKernel ring_kernel_for(int es, int mode) {
+  return es == 4 ? ring_kernel_mode<float>(mode) : ring_kernel_mode<uint16_t>(mode);
+}
+
+}  // namespace
+
+int ce_ring_smem_bytes() { return kRingHdrBytes + kRingSlots * kRingPieceBytes; }
+
+gh_status_t ce_ring_launch(const CeArgs& a, int es, int grid, cudaStream_t stream) {
+  if (a.mode != kModeFwd && a.mode != kModeSelect) return GH_ERR_INVALID_ARG;
+  const RingKernel kern = ring_kernel_for(es, a.mode);
+  static bool raised[64][2][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GH_ERR_CUDA;
+  const int kv = es == 4, km = a.mode == kModeSelect;
+  if (dev < 64 && !raised[dev][kv][km]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, ce_ring_smem_bytes()) !=
+        cudaSuccess)
+      return GH_ERR_CUDA;
+    raised[dev][kv][km] = true;
+  }
+  ProfileScope prof(a.profile_kind, stream);
+  note_launch();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kRingThreads), ce_ring_smem_bytes(), stream, 1,
+                    a) == cudaSuccess
+             ? GH_OK
+             : GH_ERR_CUDA;
+}
+
+}  // namespace gh
