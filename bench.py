@@ -410,6 +410,22 @@ class LinearCase:
 
 
 KERNEL_OF = {"ce": "ce_row", "linear": "logits_gemm"}
+CE_RING_MIN_ROWS_PER_SM = 8  # the library's switch from the row kernel to the ring pipelines
+
+
+def ce_kernel_of(case, device_index):
+    """(kernel name, profile summary file, its sources) of the CE kernel the
+    library picks for this batch: the ring pipelines from 8 rows per SM up,
+    the row kernel below (GH_CE_PATH overrides, as in the library)."""
+    import torch
+    sms = torch.cuda.get_device_properties(device_index).multi_processor_count
+    forced = os.environ.get("GH_CE_PATH")
+    ring = forced == "ring" or (forced != "rows" and case.p.B >= CE_RING_MIN_ROWS_PER_SM * sms)
+    common = ["lm_head_cross_gh_b200/csrc/ce_device.cuh", "lm_head_cross_gh_b200/csrc/common.cuh"]
+    if ring:
+        name = "ce_ring2_kernel" if case.op == "fwd_bwd" else "ce_ring_kernel"
+        return name, f"{name}.md", ["lm_head_cross_gh_b200/csrc/ce_ring.cu"] + common
+    return "ce_row_kernel", "ce_row_kernel.md", ["lm_head_cross_gh_b200/csrc/ce.cu"] + common
 
 
 def time_steps(case, dist, steps, warmup, clocks=None):
@@ -573,9 +589,10 @@ def main():
         k_ms, k_n = kern["ce_row"]
         k_avg = k_ms / max(k_n, 1)
         achieved = case.bytes_per_step / (k_avg * 1e-3) / 1e9
-        digest = source_digest(["lm_head_cross_gh_b200/csrc/ce.cu", "lm_head_cross_gh_b200/csrc/common.cuh"])
-        traffic = profiled_traffic("ce_row_kernel.md", digest, case.p.name) if case.op == "fwd_bwd" else None
-        out["roofline"] = {"bound": "hbm", "kernel": "ce_row_kernel", "achieved": achieved,
+        kname, kfile, ksrc = ce_kernel_of(case, dist.local)
+        digest = source_digest(ksrc)
+        traffic = profiled_traffic(kfile, digest, case.p.name)
+        out["roofline"] = {"bound": "hbm", "kernel": kname, "achieved": achieved,
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                            "traffic": traffic, "algorithmic_bytes": case.bytes_per_step,
                            "kernel_ms": k_avg, "peak_source": f"{pk_kind} (copy)", "source_sha": digest}

@@ -800,15 +800,15 @@ gh_status_t row_plan(int64_t V, int es, CePlan* out, int64_t* active_out) {
 
 }  // namespace
 
-// Forward-only rows take the ring pipeline (ce_fwd.cu) when there are enough
-// rows to keep every SM's ring busy (round-robin rows: at least kRingMinRowsPerSm
-// per SM keeps the last wave's imbalance small); fewer rows take the row
-// kernel, whose clusters split long rows over several SMs.  GH_CE_FWD_PATH=ring
-// or =rows forces one of the two (tests).
+// Rows take the ring pipelines (ce_ring.cu) when there are enough of them to
+// keep every SM's ring busy (round-robin rows: at least kRingMinRowsPerSm per
+// SM keeps the last wave's imbalance small); fewer rows take the row kernel,
+// whose clusters split long rows over several SMs.  GH_CE_PATH=ring or =rows
+// forces one of the two (tests, measurements).
 constexpr int kRingMinRowsPerSm = 8;
 
 static bool use_ring(int64_t B, int sms) {
-  const char* e = std::getenv("GH_CE_FWD_PATH");
+  const char* e = std::getenv("GH_CE_PATH");
   if (e && std::strcmp(e, "ring") == 0) return true;
   if (e && std::strcmp(e, "rows") == 0) return false;
   return B >= static_cast<int64_t>(kRingMinRowsPerSm) * sms;
@@ -818,7 +818,7 @@ gh_status_t ce_launch(const CeArgs& args_in, int64_t B, gh_dtype_t dtype, cudaSt
   CeArgs a = args_in;
   a.B = B;
   const int es = dtype == GH_F32 ? 4 : 2;
-  if (a.mode != kModeFwdBwd) {
+  {
     const int sms = device_sm_count();
     if (use_ring(B, sms)) return ce_ring_launch(a, es, static_cast<int>(std::min<int64_t>(B, sms)), stream);
   }

@@ -48,8 +48,9 @@ CePlan ce_plan(int64_t V, int elem_bytes);
 gh_status_t ce_count_launch(const int64_t* targets, int64_t n, int64_t V, int64_t ii,
                             unsigned long long* count, cudaStream_t stream);
 gh_status_t ce_launch(const CeArgs& args, int64_t B, gh_dtype_t dtype, cudaStream_t stream);
-// Forward-only ring pipeline (ce_fwd.cu): modes kModeFwd and kModeSelect,
-// one persistent CTA per SM (`grid` CTAs), rows round-robin over the CTAs.
+// Ring pipelines (ce_ring.cu): one persistent CTA per SM (`grid` CTAs), rows
+// round-robin over the CTAs; kModeFwd / kModeSelect stream each row once,
+// kModeFwdBwd twice (the second copy from L2) and store the gradient.
 int ce_ring_smem_bytes();
 gh_status_t ce_ring_launch(const CeArgs& args, int elem_bytes, int grid, cudaStream_t stream);
 gh_status_t ce_reduce_launch(const float* row_loss, int64_t B, const unsigned long long* n_valid, int mean,

@@ -1,4 +1,4 @@
-// Device helpers shared by the cross-entropy kernels (ce.cu, ce_fwd.cu):
+// Device helpers shared by the cross-entropy kernels (ce.cu, ce_ring.cu):
 // element access for fp32 and bf16 rows, 16-byte chunk (un)packing, and the
 // online (max, sum of exponentials) state with its exact-up-to-rounding merge.
 #pragma once

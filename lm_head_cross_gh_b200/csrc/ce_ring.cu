@@ -61,7 +61,9 @@ struct RingShared {
   uint64_t empty[kRingSlots];  // piece consumed (one arrival per warp of its group)
   uint64_t rowfull[kRingFinalizers];   // per valid row k % 4: every consumer warp posted its state
   uint64_t rowempty[kRingFinalizers];  // per valid row k % 4: its finalizer has read the states
+  uint64_t lseready[kRingFinalizers];  // two-pass kernel, per valid row k % 4: lse[k % 4] is set
   float2 part[kRingFinalizers][kRingConsumerWarps];
+  float lse[kRingFinalizers];
   int abort;                   // a wait ran out: every role stops waiting
 };
 static_assert(sizeof(RingShared) <= kRingHdrBytes, "ring header too large");
@@ -363,6 +365,339 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Forward and backward: two passes over every row through the same ring.
+//
+// Pass 1 of row k is the forward kernel's (online max / sum, the finalizer
+// merges, writes the row loss and publishes lse); pass 2 of row k copies the
+// row into the ring again and stores the gradient scale (1 + 2 z lse) exp(x -
+// lse), less scale at the target, straight from registers to global.  The
+// producer interleaves the passes one row apart -- pass 1 of row k, then pass 2
+// of row k - 1 -- so lse(k - 1) is ready when its pass 2 lands and the row was
+// read from HBM one row earlier: the second copy comes from L2 (126 MB; all
+// SMs together keep about two rows each in flight).  HBM sees one read and one
+// write of every logit; every element costs two exponentials.  Ignored rows
+// skip both copies and get a zero gradient row.
+// ---------------------------------------------------------------------------
+
+// Gradient of one 16-byte chunk: element e0 + j of the row gets
+// coef 2^(x_j log2e + nl) (nl = -lse log2e), minus scale at the target (chunk
+// position tj, or -1).  `dst` is the chunk's first element in the gradient row.
+template <typename T>
+__device__ __forceinline__ void grad_chunk(const uint4& q, float coef, float nl, int tj, float scale, uint8_t* dst,
+                                           bool congruent) {
+  constexpr int EPC = 16 / Elem<T>::kBytes;
+  constexpr int ES = Elem<T>::kBytes;
+  float v[EPC], g[EPC];
+  unpack16<T>(q, v);
+  const float2 l2 = make_float2(kLog2e, kLog2e), nl2 = make_float2(nl, nl), c2 = make_float2(coef, coef);
+#pragma unroll
+  for (int j = 0; j < EPC; j += 2) {
+    const float2 y = __ffma2_rn(make_float2(v[j], v[j + 1]), l2, nl2);
+    const float2 r = __fmul2_rn(make_float2(ex2(y.x), ex2(y.y)), c2);
+    g[j] = r.x;
+    g[j + 1] = r.y;
+  }
+  if (tj >= 0) {
+#pragma unroll
+    for (int j = 0; j < EPC; ++j)
+      if (j == tj) g[j] -= scale;
+  }
+  if (congruent) {
+    __stcs(reinterpret_cast<uint4*>(dst), pack16<T>(g));
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPC; ++j) Elem<T>::store(dst + j * ES, g[j]);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
+  constexpr int ES = Elem<T>::kBytes;
+  extern __shared__ __align__(128) uint8_t smem[];
+  RingShared& sh = *reinterpret_cast<RingShared*>(smem);
+  uint8_t* ring = smem + kRingHdrBytes;
+  const int warp = static_cast<int>(threadIdx.x) >> 5, lane = static_cast<int>(threadIdx.x) & 31;
+  const int64_t G = gridDim.x;
+  const int64_t first = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRingSlots; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.empty[i], kGroupWarps);
+    }
+    for (int i = 0; i < kRingFinalizers; ++i) {
+      mbar_init(&sh.rowfull[i], kRingConsumerWarps);
+      mbar_init(&sh.rowempty[i], 1);
+      mbar_init(&sh.lseready[i], 1);
+    }
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  pdl_wait();     // the predecessor's outputs (targets, logits, n_valid) are complete
+  pdl_trigger();  // persistent grid: the next kernel may start launching
+  __syncthreads();
+
+  volatile int* abort_flag = &sh.abort;
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *abort_flag = 1;
+    return false;
+  };
+  auto target_of = [&](int64_t row) -> int64_t { return row < a.B ? a.targets[row] : int64_t(0); };
+  auto grad_row = [&](int64_t row) -> uint8_t* { return static_cast<uint8_t*>(a.grad) + row * a.ld * ES; };
+  // byte phase of a logits row within its 16-byte chunk
+  auto row_lead = [&](int64_t row) -> int {
+    return static_cast<int>((reinterpret_cast<uintptr_t>(a.logits) + static_cast<uintptr_t>(row * a.ld * ES)) & 15);
+  };
+
+  if (warp == kRingConsumerWarps) {
+    // ---------------- producer: pass 1 of row i, then pass 2 of row i - 1 ----------------
+    if (lane == 0) {
+      uint32_t n = 0;  // pieces issued
+      auto issue_row = [&](int64_t row) -> bool {
+        const RingRow r = ring_row<ES>(a, row);
+        const int np = ring_pieces(r);
+        for (int p = 0; p < np; ++p, ++n) {
+          const int s = static_cast<int>(n % kRingSlots);
+          if (!wait(&sh.empty[s], ((n / kRingSlots) & 1) ^ 1)) return false;
+          const int c0 = r.c_lo + p * kRingPieceChunks;
+          const uint32_t bytes = 16u * static_cast<uint32_t>(tmin(kRingPieceChunks, r.c_hi - c0));
+          mbar_arrive_expect_tx(&sh.full[s], bytes);
+          bulk_g2s(ring + s * kRingPieceBytes, r.base + 16 * static_cast<int64_t>(c0), bytes, &sh.full[s]);
+        }
+        return true;
+      };
+      int64_t t = target_of(first);
+      bool prev_valid = false;
+      for (int64_t row = first;; row += G) {
+        const bool has = row < a.B;
+        const int64_t t_next = has ? target_of(row + G) : 0;
+        const bool valid = has && ring_target_valid(a, t);
+        if (valid && !issue_row(row)) break;
+        if (prev_valid && !issue_row(row - G)) break;
+        if (!has || *abort_flag) break;
+        prev_valid = valid;
+        t = t_next;
+      }
+      if (*abort_flag) {  // the copies still in flight land before the CTA exits
+        for (uint32_t k = (n > kRingSlots ? n - kRingSlots : 0); k < n; ++k)
+          (void)mbar_wait(&sh.full[k % kRingSlots], (k / kRingSlots) & 1);
+      }
+    }
+    return;
+  }
+
+  const unsigned long long nv = *a.n_valid;
+  const float scale = a.mean ? 1.0f / static_cast<float>(nv > 0 ? nv : 1ull) : 1.0f;
+
+  if (warp > kRingConsumerWarps) {
+    // ---------------- finalizers ----------------
+    const uint32_t f = warp - kRingConsumerWarps - 1;
+    uint32_t k = 0;  // valid rows seen
+    uint32_t i = 0;  // rows seen
+    int64_t t = target_of(first);
+    for (int64_t row = first; row < a.B; row += G, ++i) {
+      const int64_t t_next = target_of(row + G);
+      if (!ring_target_valid(a, t)) {
+        if (lane == 0 && i % kRingFinalizers == f) a.row_loss[row] = 0.0f;
+        t = t_next;
+        continue;
+      }
+      if (k % kRingFinalizers != f) {
+        ++k;
+        t = t_next;
+        continue;
+      }
+      const RingRow r = ring_row<ES>(a, row);
+      const uint8_t* src = static_cast<const uint8_t*>(a.logits) + row * a.ld * ES;
+      // ragged ends: lanes 0-15 the head elements, lanes 16-31 the tail
+      int64_t e = -1;
+      if (lane < 16) {
+        if (lane < r.h) e = lane;
+      } else if (r.tail + (lane - 16) < a.V) {
+        e = r.tail + (lane - 16);
+      }
+      const float edge = e >= 0 ? Elem<T>::load(src + e * ES) : kNegInf;
+      const float xt = Elem<T>::load(src + t * ES);
+      const int j = static_cast<int>(f);
+      const bool ok = __all_sync(0xffffffffu, wait(&sh.rowfull[j], (k / kRingFinalizers) & 1));
+      MaxSum st = (lane < kRingConsumerWarps && ok) ? MaxSum{sh.part[j][lane].x, sh.part[j][lane].y}
+                                                    : MaxSum{kNegInf, 0.0f};
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.rowempty[j]);
+      st = combine(st, edge == kNegInf ? MaxSum{kNegInf, 0.0f} : MaxSum{edge, 1.0f});
+      st = warp_reduce(st);
+      const float lse = st.m + logf(st.s);
+      if (lane == 0) {
+        sh.lse[j] = lse;
+        mbar_arrive(&sh.lseready[j]);
+        a.row_loss[row] = (lse - xt) + a.z * lse * lse;
+      }
+      if (e >= 0) {  // the ragged ends' gradient
+        const float coef = scale * (1.0f + 2.0f * a.z * lse);
+        float g = coef * ex2(fmaf(edge, kLog2e, -lse * kLog2e));
+        if (e == t) g -= scale;
+        Elem<T>::store(grad_row(row) + e * ES, g);
+      }
+      ++k;
+      t = t_next;
+      if (!ok) break;
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int grp = warp / kGroupWarps;
+  const int gtid = static_cast<int>(threadIdx.x) - grp * kGroupThreads;
+  const int tid = static_cast<int>(threadIdx.x);
+  uint32_t n = 0;  // pieces seen (this group consumes n % kRingGroups == grp)
+  uint32_t k = 0;  // valid rows seen
+  bool ok = true;
+
+  // pass 1 of a valid row: the online (max, sum) state, posted for the finalizer
+  auto pass1 = [&](int64_t row) {
+    const RingRow r = ring_row<ES>(a, row);
+    const int np = ring_pieces(r);
+    const int nbc = r.c_hi - r.c_lo;
+    MaxSum st{kNegInf, 0.0f};
+    for (int p = 0; p < np; ++p, ++n) {
+      if (static_cast<int>(n % kRingGroups) != grp) continue;
+      const int s = static_cast<int>(n % kRingSlots);
+      if (!__all_sync(0xffffffffu, wait(&sh.full[s], (n / kRingSlots) & 1))) {
+        ok = false;
+        return;
+      }
+      const uint8_t* piece = ring + s * kRingPieceBytes;
+      const int nc = tmin(kRingPieceChunks, nbc - p * kRingPieceChunks);
+      if (nc == kRingPieceChunks) {
+        uint4 q[kPieceChunksPerThread];
+#pragma unroll
+        for (int i = 0; i < kPieceChunksPerThread; ++i)
+          q[i] = *reinterpret_cast<const uint4*>(piece + 16 * (gtid + i * kGroupThreads));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
+        fold_full_piece<T>(st, q);
+      } else {
+        for (int c = gtid; c < nc; c += kGroupThreads) fold_one<T>(st, *reinterpret_cast<const uint4*>(piece + 16 * c));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
+      }
+    }
+    st = warp_reduce(st);
+    const int j = static_cast<int>(k % kRingFinalizers);
+    if (lane == 0) {
+      if (wait(&sh.rowempty[j], ((k / kRingFinalizers) & 1) ^ 1)) {
+        sh.part[j][warp] = make_float2(st.m, st.s);
+        mbar_arrive(&sh.rowfull[j]);
+      }
+    }
+    __syncwarp();
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) ok = false;
+  };
+
+  // pass 2 of valid row `row` (valid-row index kr, target t): the gradient of
+  // its whole chunks
+  auto pass2 = [&](int64_t row, int64_t t, uint32_t kr) {
+    const RingRow r = ring_row<ES>(a, row);
+    const int np = ring_pieces(r);
+    const int nbc = r.c_hi - r.c_lo;
+    const int j = static_cast<int>(kr % kRingFinalizers);
+    // every consumer warp waits for every row's lse, so each lseready phase is
+    // observed in order
+    if (!__all_sync(0xffffffffu, wait(&sh.lseready[j], (kr / kRingFinalizers) & 1))) {
+      ok = false;
+      return;
+    }
+    const float lse = sh.lse[j];
+    const float coef = scale * (1.0f + 2.0f * a.z * lse);
+    const float nl = -lse * kLog2e;
+    const int lead = row_lead(row);
+    uint8_t* gbase = grad_row(row) - lead;  // chunk c's gradient bytes start at gbase + 16 c
+    const bool congruent = a.congruent != 0;
+    const int64_t tb = lead + t * ES;        // target's byte in the row's chunk space
+    const int tc = static_cast<int>(tb >> 4), tj = static_cast<int>((tb & 15) / ES);
+    for (int p = 0; p < np; ++p, ++n) {
+      if (static_cast<int>(n % kRingGroups) != grp) continue;
+      const int s = static_cast<int>(n % kRingSlots);
+      if (!__all_sync(0xffffffffu, wait(&sh.full[s], (n / kRingSlots) & 1))) {
+        ok = false;
+        return;
+      }
+      const uint8_t* piece = ring + s * kRingPieceBytes;
+      const int c0 = r.c_lo + p * kRingPieceChunks;
+      const int nc = tmin(kRingPieceChunks, nbc - p * kRingPieceChunks);
+      if (nc == kRingPieceChunks) {
+        uint4 q[kPieceChunksPerThread];
+#pragma unroll
+        for (int i = 0; i < kPieceChunksPerThread; ++i)
+          q[i] = *reinterpret_cast<const uint4*>(piece + 16 * (gtid + i * kGroupThreads));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
+#pragma unroll
+        for (int i = 0; i < kPieceChunksPerThread; ++i) {
+          const int c = c0 + gtid + i * kGroupThreads;
+          grad_chunk<T>(q[i], coef, nl, c == tc ? tj : -1, scale, gbase + 16 * static_cast<int64_t>(c), congruent);
+        }
+      } else {
+        for (int cc = gtid; cc < nc; cc += kGroupThreads) {
+          const int c = c0 + cc;
+          grad_chunk<T>(*reinterpret_cast<const uint4*>(piece + 16 * cc), coef, nl, c == tc ? tj : -1, scale,
+                        gbase + 16 * static_cast<int64_t>(c), congruent);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
+      }
+    }
+  };
+
+  // an ignored row: zero gradient (whole chunks and ragged ends), no copies
+  auto zero_row = [&](int64_t row) {
+    const RingRow r = ring_row<ES>(a, row);
+    uint8_t* g = grad_row(row);
+    uint8_t* gbase = g - row_lead(row);
+    if (a.congruent) {
+      for (int c = r.c_lo + tid; c < r.c_hi; c += kRingConsumers)
+        __stcs(reinterpret_cast<uint4*>(gbase + 16 * static_cast<int64_t>(c)), make_uint4(0, 0, 0, 0));
+    } else {
+      for (int64_t e = r.h + tid; e < r.tail; e += kRingConsumers) Elem<T>::store(g + e * ES, 0.0f);
+    }
+    if (tid < r.h) Elem<T>::store(g + static_cast<int64_t>(tid) * ES, 0.0f);
+    if (tid >= 32 && tid < 48 && r.tail + (tid - 32) < a.V) Elem<T>::store(g + (r.tail + (tid - 32)) * ES, 0.0f);
+  };
+
+  int64_t t = target_of(first);
+  bool prev_valid = false;
+  int64_t prev_t = 0;
+  uint32_t prev_k = 0;
+  for (int64_t row = first;; row += G) {
+    const bool has = row < a.B;
+    const int64_t t_next = has ? target_of(row + G) : 0;
+    const bool valid = has && ring_target_valid(a, t);
+    const uint32_t kr = k;
+    if (valid) {
+      pass1(row);
+      ++k;
+      if (!ok) break;
+    }
+    if (row - G >= first) {  // pass 2 (or the zero row) of the previous row
+      if (prev_valid) {
+        pass2(row - G, prev_t, prev_k);
+        if (!ok) break;
+      } else {
+        zero_row(row - G);
+      }
+    }
+    if (!has) break;
+    prev_valid = valid;
+    prev_t = t;
+    prev_k = kr;
+    t = t_next;
+  }
+}
+
 using RingKernel = void (*)(CeArgs);
 
 template <typename T>
@@ -379,12 +714,12 @@ RingKernel ring_kernel_for(int es, int mode) {
 int ce_ring_smem_bytes() { return kRingHdrBytes + kRingSlots * kRingPieceBytes; }
 
 gh_status_t ce_ring_launch(const CeArgs& a, int es, int grid, cudaStream_t stream) {
-  if (a.mode != kModeFwd && a.mode != kModeSelect) return GH_ERR_INVALID_ARG;
-  const RingKernel kern = ring_kernel_for(es, a.mode);
-  static bool raised[64][2][2] = {};
+  const RingKernel kern = a.mode == kModeFwdBwd ? (es == 4 ? ce_ring2_kernel<float> : ce_ring2_kernel<uint16_t>)
+                                                : ring_kernel_for(es, a.mode);
+  static bool raised[64][2][3] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GH_ERR_CUDA;
-  const int kv = es == 4, km = a.mode == kModeSelect;
+  const int kv = es == 4, km = a.mode;
   if (dev < 64 && !raised[dev][kv][km]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, ce_ring_smem_bytes()) !=
         cudaSuccess)

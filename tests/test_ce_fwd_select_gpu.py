@@ -5,7 +5,7 @@ Two kernels serve both calls: the row kernel in a forward-only mode (one CTA
 per row, a cluster of CTAs per long row, the two-pass streaming kernel beyond
 that; the default below 8 rows per SM) and the ring pipeline (pieces of rows
 streamed through a shared-memory ring; the default from 8 rows per SM up).
-The `path` fixture runs each case on both (GH_CE_FWD_PATH); the ring's own
+The `path` fixture runs each case on both (GH_CE_PATH); the ring's own
 cases cover every 16-byte phase of a row's start, rows without a whole
 16-byte chunk and rows of many pieces.
 
@@ -35,7 +35,7 @@ def path(request, monkeypatch):
     """Both forward-only kernels: the row kernel (clusters for long rows, the
     streaming kernel beyond them) and the ring pipeline (the default from
     8 rows per SM up)."""
-    monkeypatch.setenv("GH_CE_FWD_PATH", request.param)
+    monkeypatch.setenv("GH_CE_PATH", request.param)
     return request.param
 
 
@@ -209,7 +209,7 @@ def test_ring_row_alignments_and_tiny_rows(cuda_device, dtype):
 
 
 def test_ring_many_pieces_per_row(cuda_device, monkeypatch):
-    monkeypatch.setenv("GH_CE_FWD_PATH", "ring")
+    monkeypatch.setenv("GH_CE_PATH", "ring")
     # 262147 bf16 = 33 pieces of 16 KiB; more pieces per CTA than ring slots
     p = gh_synth.ce_student_t_spiked(200, 262147, dtype="bf16", reduction="mean", z_loss=1e-4, seed=31)
     check_fwd(p, *fwd(p), "ring spiked 262147")

@@ -1,8 +1,9 @@
 """GPU parity of gh_ce_fwd_bwd against the float64 oracle (through the C ABI).
 
 Covers the small fp32 workload, ragged vocabulary sizes around every vector and
-chunk boundary, all three kernel paths (one CTA per row, a cluster of CTAs per
-row, the two-pass streaming path for very long rows), in-place gradients, a
+chunk boundary, every kernel path (one CTA per row, a cluster of CTAs per row,
+the two-pass streaming path for very long rows, and the two-pass ring pipeline,
+each case run on the row kernel and on the ring), in-place gradients, a
 gradient buffer whose 16-byte phase differs from the logits', ignored and
 out-of-range targets, determinism, and the full-size GPT-2 and large-vocabulary
 workloads on sampled rows.
@@ -19,6 +20,15 @@ import oracle
 from ce_check import check_grad, check_loss, check_problem_full, grad_to_f64, loss_atol, row_eps, to_device
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, params=["rows", "ring"])
+def ce_path(request, monkeypatch):
+    """Every case on both forward+backward kernels: the row kernel (a row, or a
+    cluster's slices of it, resident in shared memory; the two-pass streaming
+    kernel beyond) and the two-pass ring pipeline (the second pass from L2)."""
+    monkeypatch.setenv("GH_CE_PATH", request.param)
+    return request.param
 
 
 def run(p, **kw):
