@@ -59,18 +59,19 @@ def source_digest(files):
     return h.hexdigest()[:12]
 
 
-def profiled_traffic(summary_file, digest, workload):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
-    p = os.path.join(ROOT, "profiles", summary_file)
-    if not os.path.exists(p):
-        return None
-    txt = open(p).read()
-    m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", txt)
-    m_wl = re.search(r"workload:\s*(\S+)", txt)
-    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
-    if not (m_sha and m_tr and m_wl) or m_sha.group(1) != digest or m_wl.group(1) != workload:
-        return None
-    return float(m_tr.group(1))
+def profiled_traffic(kernel, digest, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu summary
+    (`profiles/<kernel>_*.md`), if one was taken of the current source."""
+    import glob
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*.md"))):
+        txt = open(p).read()
+        m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", txt)
+        if not m_sha or m_sha.group(1) != digest:
+            continue
+        for m in re.finditer(r"workload:\s*(\S+)\s*\ntraffic_bytes_per_launch:\s*([0-9.eE+]+)", txt):
+            if m.group(1) == workload:
+                return float(m.group(2))
+    return None
 
 
 # --------------------------------------------------------------------------
@@ -414,7 +415,7 @@ CE_RING_MIN_ROWS_PER_SM = 8  # the library's switch from the row kernel to the r
 
 
 def ce_kernel_of(case, device_index):
-    """(kernel name, profile summary file, its sources) of the CE kernel the
+    """(kernel name, its sources) of the CE kernel the
     library picks for this batch: the ring pipelines from 8 rows per SM up,
     the row kernel below (GH_CE_PATH overrides, as in the library)."""
     import torch
@@ -424,8 +425,8 @@ def ce_kernel_of(case, device_index):
     common = ["lm_head_cross_gh_b200/csrc/ce_device.cuh", "lm_head_cross_gh_b200/csrc/common.cuh"]
     if ring:
         name = "ce_ring2_kernel" if case.op == "fwd_bwd" else "ce_ring_kernel"
-        return name, f"{name}.md", ["lm_head_cross_gh_b200/csrc/ce_ring.cu"] + common
-    return "ce_row_kernel", "ce_row_kernel.md", ["lm_head_cross_gh_b200/csrc/ce.cu"] + common
+        return name, ["lm_head_cross_gh_b200/csrc/ce_ring.cu"] + common
+    return "ce_row_kernel", ["lm_head_cross_gh_b200/csrc/ce.cu"] + common
 
 
 def time_steps(case, dist, steps, warmup, clocks=None):
@@ -589,9 +590,9 @@ def main():
         k_ms, k_n = kern["ce_row"]
         k_avg = k_ms / max(k_n, 1)
         achieved = case.bytes_per_step / (k_avg * 1e-3) / 1e9
-        kname, kfile, ksrc = ce_kernel_of(case, dist.local)
+        kname, ksrc = ce_kernel_of(case, dist.local)
         digest = source_digest(ksrc)
-        traffic = profiled_traffic(kfile, digest, case.p.name)
+        traffic = profiled_traffic(kname, digest, case.p.name)
         out["roofline"] = {"bound": "hbm", "kernel": kname, "achieved": achieved,
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                            "traffic": traffic, "algorithmic_bytes": case.bytes_per_step,
