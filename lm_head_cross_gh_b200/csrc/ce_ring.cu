@@ -13,11 +13,11 @@
 //                        thread loads its eight chunks into registers, the
 //                        group frees the slot at once, and the thread folds the
 //                        chunks into its online (max, sum of exp) state;
-//                        at a row's end each warp reduces its state and posts
-//                        it to the row's finalizer;
+//                        at a row's end each thread posts its state to the
+//                        row's finalizer (no reduction on the consumers);
 //   warps 17-20 (finalizers)
 //                        take the valid rows in turn (row k to warp 17 + k % 4);
-//                        each merges the 16 warp states with the row's ragged
+//                        each merges the 512 thread states with the row's ragged
 //                        ends (the elements outside the whole 16-byte chunks,
 //                        read from global), reads the target logit and writes
 //                        the row value.  With four of them, a finalizer's
@@ -54,7 +54,7 @@ constexpr int kRingPieceChunks = kRingPieceBytes / 16;
 constexpr int kPieceChunksPerThread = kRingPieceChunks / kGroupThreads;  // 8
 static_assert(kRingSlots % kRingGroups == 0, "a slot always serves the same group");
 static_assert(kRingPieceChunks % kGroupThreads == 0, "whole chunks per thread");
-constexpr int kRingHdrBytes = 1024;
+constexpr int kRingHdrBytes = 17408;  // barriers, 4 x 512 row states, lse
 
 struct RingShared {
   uint64_t full[kRingSlots];   // piece landed (producer's expect_tx + the copy's bytes)
@@ -62,7 +62,7 @@ struct RingShared {
   uint64_t rowfull[kRingFinalizers];   // per valid row k % 4: every consumer warp posted its state
   uint64_t rowempty[kRingFinalizers];  // per valid row k % 4: its finalizer has read the states
   uint64_t lseready[kRingFinalizers];  // two-pass kernel, per valid row k % 4: lse[k % 4] is set
-  float2 part[kRingFinalizers][kRingConsumerWarps];
+  float2 part[kRingFinalizers][kRingConsumerWarps][32];  // every consumer thread's row state
   float lse[kRingFinalizers];
   int abort;                   // a wait ran out: every role stops waiting
 };
@@ -97,6 +97,26 @@ __device__ __forceinline__ int ring_pieces(const RingRow& r) {
 
 __device__ __forceinline__ bool ring_target_valid(const CeArgs& a, int64_t t) {
   return (t != a.ignore_index) && t >= 0 && t < a.V;
+}
+
+// A finalizer lane's share of a row's merge: the states consumer lane `lane`
+// of each of the 16 consumer warps posted (max first, then one rescale each).
+__device__ __forceinline__ MaxSum merge_lane_states(const float2 (*part)[32], int lane) {
+  float m[kRingConsumerWarps], sv[kRingConsumerWarps];
+  float M = kNegInf;
+#pragma unroll
+  for (int w = 0; w < kRingConsumerWarps; ++w) {
+    const float2 v = part[w][lane];
+    m[w] = v.x;
+    sv[w] = v.y;
+    M = fmaxf(M, v.x);
+  }
+  if (M == kNegInf) return {kNegInf, 0.0f};
+  float S = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kRingConsumerWarps; ++w)
+    if (m[w] != kNegInf) S += sv[w] * ex2((m[w] - M) * kLog2e);
+  return {M, S};
 }
 
 // The running reference of a thread's online sum is its max so far plus
@@ -290,8 +310,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
       const float xt = Elem<T>::load(src + t * ES);
       const int j = static_cast<int>(f);
       const bool ok = __all_sync(0xffffffffu, wait(&sh.rowfull[j], (k / kRingFinalizers) & 1));
-      MaxSum st = (lane < kRingConsumerWarps && ok) ? MaxSum{sh.part[j][lane].x, sh.part[j][lane].y}
-                                                    : MaxSum{kNegInf, 0.0f};
+      MaxSum st = ok ? merge_lane_states(sh.part[j], lane) : MaxSum{kNegInf, 0.0f};
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.rowempty[j]);
       st = combine(st, edge == kNegInf ? MaxSum{kNegInf, 0.0f} : MaxSum{edge, 1.0f});
@@ -308,6 +327,20 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
   }
 
   // ---------------- consumers ----------------
+  // Each thread posts its own (max, sum) state of valid row k for the row's
+  // finalizer (no reduction here: the finalizer merges the 512 states).
+  auto post_state = [&](const MaxSum& st, uint32_t k) {
+    const int j = static_cast<int>(k % kRingFinalizers);
+    bool free_slot = true;
+    if (lane == 0) free_slot = wait(&sh.rowempty[j], ((k / kRingFinalizers) & 1) ^ 1);
+    __syncwarp();
+    if (__shfl_sync(0xffffffffu, free_slot ? 1 : 0, 0)) {
+      sh.part[j][warp][lane] = make_float2(st.m, st.s);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.rowfull[j]);
+    }
+    __syncwarp();
+  };
   const int grp = warp / kGroupWarps;
   const int gtid = static_cast<int>(threadIdx.x) - grp * kGroupThreads;
   uint32_t n = 0;  // pieces seen (this group consumes n % kRingGroups == grp)
@@ -350,15 +383,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
       }
     }
     if (!ok) break;
-    st = warp_reduce(st);
-    const int j = static_cast<int>(k % kRingFinalizers);
-    if (lane == 0) {
-      if (wait(&sh.rowempty[j], ((k / kRingFinalizers) & 1) ^ 1)) {
-        sh.part[j][warp] = make_float2(st.m, st.s);
-        mbar_arrive(&sh.rowfull[j]);
-      }
-    }
-    __syncwarp();
+    post_state(st, k);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
     ++k;
     t = t_next;
@@ -524,8 +549,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
       const float xt = Elem<T>::load(src + t * ES);
       const int j = static_cast<int>(f);
       const bool ok = __all_sync(0xffffffffu, wait(&sh.rowfull[j], (k / kRingFinalizers) & 1));
-      MaxSum st = (lane < kRingConsumerWarps && ok) ? MaxSum{sh.part[j][lane].x, sh.part[j][lane].y}
-                                                    : MaxSum{kNegInf, 0.0f};
+      MaxSum st = ok ? merge_lane_states(sh.part[j], lane) : MaxSum{kNegInf, 0.0f};
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.rowempty[j]);
       st = combine(st, edge == kNegInf ? MaxSum{kNegInf, 0.0f} : MaxSum{edge, 1.0f});
@@ -550,6 +574,20 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
   }
 
   // ---------------- consumers ----------------
+  // Each thread posts its own (max, sum) state of valid row k for the row's
+  // finalizer (no reduction here: the finalizer merges the 512 states).
+  auto post_state = [&](const MaxSum& st, uint32_t k) {
+    const int j = static_cast<int>(k % kRingFinalizers);
+    bool free_slot = true;
+    if (lane == 0) free_slot = wait(&sh.rowempty[j], ((k / kRingFinalizers) & 1) ^ 1);
+    __syncwarp();
+    if (__shfl_sync(0xffffffffu, free_slot ? 1 : 0, 0)) {
+      sh.part[j][warp][lane] = make_float2(st.m, st.s);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.rowfull[j]);
+    }
+    __syncwarp();
+  };
   const int grp = warp / kGroupWarps;
   const int gtid = static_cast<int>(threadIdx.x) - grp * kGroupThreads;
   const int tid = static_cast<int>(threadIdx.x);
@@ -586,15 +624,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
         if (lane == 0) mbar_arrive(&sh.empty[s]);
       }
     }
-    st = warp_reduce(st);
-    const int j = static_cast<int>(k % kRingFinalizers);
-    if (lane == 0) {
-      if (wait(&sh.rowempty[j], ((k / kRingFinalizers) & 1) ^ 1)) {
-        sh.part[j][warp] = make_float2(st.m, st.s);
-        mbar_arrive(&sh.rowfull[j]);
-      }
-    }
-    __syncwarp();
+    post_state(st, k);
     if (__any_sync(0xffffffffu, *abort_flag != 0)) ok = false;
   };
 
