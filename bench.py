@@ -13,9 +13,9 @@ Timing: CUDA events on the launching stream around exactly K steps, bracketed
 by a barrier and a device synchronise, max over ranks.  Inputs are larger than
 L2 (126 MB) for the timed workloads, so no flush runs between steps.  Kernel
 durations for the roofline come from libgh's own event pairs around the
-dominant kernel, recorded over a second run of the same K steps (event
-records between kernels would hide the programmatic launch overlap, so they
-stay out of the region that gives `value`).  With N > 1 each rank
+dominant kernel, recorded over a separate run of the same K steps just before
+the timed region (event records between kernels would hide the programmatic
+launch overlap, so they stay out of the region that gives `value`).  With N > 1 each rank
 processes its own batch (seed = rank); nothing is exchanged (weak scaling).
 ``--impl reference`` times the float64 CPU oracle on a bounded sample of the
 same workload (rank 0 only).
@@ -61,7 +61,8 @@ def source_digest(files):
 
 def profiled_traffic(kernel, digest, workload):
     """DRAM bytes per launch of `kernel` on `workload` from a committed ncu summary
-    (`profiles/<kernel>_*.md`), if one was taken of the current source."""
+    (`profiles/<kernel>_*.md`; for the forward ring `<kernel>` names the
+    operation too), if one was taken of the current source."""
     import glob
     for p in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*.md"))):
         txt = open(p).read()
@@ -430,10 +431,14 @@ def ce_kernel_of(case, device_index):
 
 
 def time_steps(case, dist, steps, warmup, clocks=None):
-    """Time exactly `steps` steps (value), then the same steps again with libgh's
-    per-kernel events on (kernel durations for the roofline; the event records
-    between kernels would hide the launch overlap, so they stay out of the
-    first region)."""
+    """Kernel durations for the roofline, then exactly `steps` timed steps.
+
+    The kernel pass runs the same `steps` steps with libgh's per-kernel event
+    pairs on (one pass fills the library's event pool, the next is read); it
+    comes right after the warm-up so it sees the same clocks as the timed
+    region.  The timed region that gives `value` has no per-kernel events
+    (event records between kernels would hide the programmatic launch overlap).
+    """
     import torch
     import lm_head_cross_gh_b200 as gh
     for _ in range(warmup):
@@ -441,7 +446,16 @@ def time_steps(case, dist, steps, warmup, clocks=None):
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     kinds = ["ce_row"] if case.kind == "ce" else ["logits_gemm", "chunk_ce", "dx_gemm", "dw_gemm"]
+    for rep in range(2):
+        gh.gh_profile_enable(True)
+        for _ in range(steps):
+            case.step()
+        torch.cuda.synchronize()
     gh.gh_profile_enable(False)
+    kern = {}
+    for k in kinds:
+        tot, n = gh.gh_profile_read(k)
+        kern[k] = (tot, n)
     n0 = gh.gh_launch_count()
     if clocks:
         clocks.start()
@@ -467,17 +481,6 @@ def time_steps(case, dist, steps, warmup, clocks=None):
             torch.cuda.synchronize()
         clocks.stop()
     ms = e0.elapsed_time(e1)
-    # kernel durations: one profiled pass fills libgh's event pool, the next is read
-    for rep in range(2):
-        gh.gh_profile_enable(True)
-        for _ in range(steps):
-            case.step()
-        torch.cuda.synchronize()
-    gh.gh_profile_enable(False)
-    kern = {}
-    for k in kinds:
-        tot, n = gh.gh_profile_read(k)
-        kern[k] = (tot, n)
     return ms, launches, kern
 
 
@@ -592,7 +595,8 @@ def main():
         achieved = case.bytes_per_step / (k_avg * 1e-3) / 1e9
         kname, ksrc = ce_kernel_of(case, dist.local)
         digest = source_digest(ksrc)
-        traffic = profiled_traffic(kname, digest, case.p.name)
+        prefix = kname if kname != "ce_ring_kernel" else f"ce_ring_kernel_{case.op}"
+        traffic = profiled_traffic(prefix, digest, case.p.name)
         out["roofline"] = {"bound": "hbm", "kernel": kname, "achieved": achieved,
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                            "traffic": traffic, "algorithmic_bytes": case.bytes_per_step,

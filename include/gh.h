@@ -12,6 +12,10 @@
  *    viv `gpt_loss`), optionally unreduced.
  *  - gh_selective_log_softmax: `selective_log_softmax` — one log-probability
  *    per row, x[index] - logsumexp(x), without the full log-softmax.
+ *  - gh_ce_vjp: nuvec `FastOp::CrossEntropyVjp` — the logits gradient for a
+ *    per-row upstream gradient, from the forward's row loss.
+ *  - gh_chunked_linear_loss: `chunked_linear_loss` — the chunk loop of
+ *    gh_linear_ce with a caller-provided loss and logits gradient per chunk.
  *  - gh_linear_ce: `chunked_linear_cross_entropy` — logits = inputs @ weight.T
  *    computed one row chunk at a time and never materialised in full; per
  *    chunk the logits gradient G gives grad_inputs[chunk] = G @ weight and
@@ -145,6 +149,26 @@ gh_status_t gh_ce_fwd(const void* logits, const int64_t* targets, int64_t B, int
                       float z_mult, float* loss, float* row_loss, void* stream);
 
 /*
+ * gh_ce_vjp — the logits gradient of the per-row cross-entropy for an upstream
+ * gradient per row (nuvec FastOp::CrossEntropyVjp: logits, targets, the
+ * forward's row loss and g):
+ *     grad_j = g_r (exp(x_j - lse_r) - [j == t_r]),   lse_r = row_loss_r + x_{r,t_r}
+ * The forward's row loss carries lse, so the gradient is one streaming pass
+ * with no reduction.
+ *
+ *   logits, targets, B, V, dtype, ignore_index  as for gh_ce_fwd_bwd.
+ *   row_loss  [B] float32, device: lse - x_t per row without z-loss, as
+ *             gh_ce_fwd returns with z_mult = 0 (values of ignored rows are
+ *             not read).
+ *   g         [B] float32, device: the upstream gradient of each row's loss.
+ *   grad      [B, V] of `dtype`, device, written; grad == logits is allowed.
+ * Rows whose target equals ignore_index get a zero gradient row; a target
+ * outside [0, V) likewise, and records GH_ERR_TARGET_RANGE.  No scratch.
+ */
+gh_status_t gh_ce_vjp(const void* logits, const int64_t* targets, int64_t B, int64_t V, gh_dtype_t dtype,
+                      int64_t ignore_index, const float* row_loss, const float* g, void* grad, void* stream);
+
+/*
  * gh_selective_log_softmax — Greyhound `selective_log_softmax`: for each row
  * r, out[r] = x[r, index[r]] - logsumexp(x[r, :]), the log-probability of one
  * selected class, without materialising the log-probabilities.
@@ -186,6 +210,35 @@ gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* 
                          float* loss, void* grad_inputs, void* grad_weight, void* stream);
 
 /*
+ * gh_chunked_linear_loss — Greyhound `chunked_linear_loss`: the chunked
+ * linear projection of gh_linear_ce with a caller-provided loss in place of
+ * the cross-entropy.  For each chunk of rows [row0, row0 + rows) the library
+ * computes logits = inputs[chunk] @ weight.T into a bf16 buffer and calls
+ * `loss_fn` on the calling host thread; `loss_fn` must enqueue on `stream`
+ * (it may not wait for it) the work that
+ *   - overwrites the logits in place with the logits gradient (bf16, same
+ *     layout: row r at logits + r * ld elements, V valid columns), and
+ *   - adds the chunk's scalar loss to the float32 device scalar `loss_accum`,
+ * and return GH_OK.  The library then forms grad_inputs[chunk] = G @ weight and
+ * accumulates grad_weight (+)= G^T @ inputs[chunk] as gh_linear_ce does.
+ * The returned loss is the sum of the chunks' losses.  Slicing the caller's
+ * per-row arguments to [row0, row0 + rows) is up to `loss_fn` (`ctx`).
+ *
+ *   inputs, weight, N, D, V, chunk, accum_dtype, grad_inputs, grad_weight,
+ *   stream   as for gh_linear_ce.
+ *   loss_fn  the callback; ctx is passed through unchanged.
+ *   loss     device float32 scalar, written (0 before the first chunk).
+ * A status other than GH_OK from loss_fn stops the chunk loop; the library
+ * frees its scratch (stream-ordered) and returns that status.
+ */
+typedef gh_status_t (*gh_chunk_loss_fn)(void* ctx, int64_t row0, int64_t rows, void* logits, int64_t ld,
+                                        int64_t V, float* loss_accum, void* stream);
+
+gh_status_t gh_chunked_linear_loss(const void* inputs, const void* weight, int64_t N, int64_t D, int64_t V,
+                                   int64_t chunk, gh_accum_t accum_dtype, gh_chunk_loss_fn loss_fn, void* ctx,
+                                   float* loss, void* grad_inputs, void* grad_weight, void* stream);
+
+/*
  * gh_get_device_status — synchronises `stream`, returns the first error any
  * kernel recorded on the current device since the last call (GH_OK if none:
  * GH_ERR_TARGET_RANGE or GH_ERR_TIMEOUT), and clears it.  Returns GH_ERR_CUDA
@@ -202,7 +255,8 @@ typedef enum {
   GH_KERNEL_CHUNK_CE = 2,      /* linear-CE: per-chunk loss and logits gradient */
   GH_KERNEL_DX_GEMM = 3,       /* linear-CE: grad_inputs[chunk] = G_c @ W */
   GH_KERNEL_DW_GEMM = 4,       /* linear-CE: grad_weight (+)= G_c^T @ X_c */
-  GH_KERNEL_KINDS = 5
+  GH_KERNEL_CE_VJP = 5,        /* gh_ce_vjp */
+  GH_KERNEL_KINDS = 6
 } gh_kernel_t;
 
 /* gh_profile_enable(1) discards earlier records and starts recording a pair

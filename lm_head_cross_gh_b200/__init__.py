@@ -46,6 +46,10 @@ class GhError(RuntimeError):
 
 _lib = None
 
+# gh_chunk_loss_fn(ctx, row0, rows, logits, ld, V, loss_accum, stream) -> gh_status_t
+CHUNK_LOSS_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                 ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p)
+
 
 def lib() -> ctypes.CDLL:
     """The loaded ``libgh.so`` with argument types set (loads on first use)."""
@@ -66,6 +70,12 @@ def lib() -> ctypes.CDLL:
     L.gh_ce_fwd.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_int, c_float,
                             c_void_p, c_void_p, c_void_p]
     L.gh_ce_fwd.restype = c_int
+    L.gh_chunked_linear_loss.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int,
+                                         CHUNK_LOSS_FN, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
+    L.gh_chunked_linear_loss.restype = c_int
+    L.gh_ce_vjp.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_void_p, c_void_p, c_void_p,
+                            c_void_p]
+    L.gh_ce_vjp.restype = c_int
     L.gh_selective_log_softmax.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_void_p, c_void_p]
     L.gh_selective_log_softmax.restype = c_int
     L.gh_linear_ce.argtypes = [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int,
@@ -92,6 +102,7 @@ def header_symbols() -> list:
     with open(HEADER_PATH) as f:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"\btypedef\b[^;]*;", "", text, flags=re.S)  # enums and the callback type
     return sorted(set(re.findall(r"\b(gh_[a-z0-9_]+)\s*\(", text)))
 
 
@@ -218,6 +229,102 @@ def gh_ce_fwd(logits, targets, ignore_index: int = -100, reduction: str = "mean"
     return loss, row_loss
 
 
+class _DeviceView:
+    """A CUDA array interface over memory the library owns during a callback."""
+
+    def __init__(self, ptr, shape, strides, typestr):
+        self.__cuda_array_interface__ = {"version": 3, "data": (ptr, False), "shape": tuple(shape),
+                                         "strides": tuple(strides), "typestr": typestr, "stream": None}
+
+
+def gh_chunked_linear_loss(inputs, weight, loss_and_grad_fn, *loss_args, chunk: int = 0, accum: str = "fp32",
+                           grad_inputs=None, grad_weight=None, loss=None, stream=None, **loss_kwargs):
+    """Chunked linear projection with a caller-provided loss (``gh_chunked_linear_loss``).
+
+    For each row chunk the library computes ``logits = inputs[c] @ weight.T``
+    (bf16) and this wrapper calls ``loss_and_grad_fn(logits_chunk, *args,
+    **kwargs)`` on the library's stream; tensor arguments whose leading
+    dimension is N are sliced to the chunk's rows.  The function returns
+    ``(loss, grad_logits)``: a scalar and a tensor shaped like the chunk.  The
+    gradient is written over the chunk logits, the loss added to the total.
+    Returns ``(loss, grad_inputs, grad_weight)``; the loss is the sum over chunks.
+    """
+    import torch
+    _need(inputs.dim() == 2 and weight.dim() == 2 and inputs.shape[1] == weight.shape[1], "shapes")
+    _need(inputs.dtype == torch.bfloat16 and weight.dtype == torch.bfloat16, "inputs/weight must be bfloat16")
+    _need(inputs.is_cuda and weight.is_cuda and inputs.is_contiguous() and weight.is_contiguous(), "layout")
+    _need(accum in GH_ACCUM, "accum must be 'fp32' or 'weight'")
+    N, D = inputs.shape
+    V = weight.shape[0]
+    dev = inputs.device
+    if grad_inputs is None:
+        grad_inputs = torch.empty_like(inputs)
+    if grad_weight is None:
+        grad_weight = torch.empty_like(weight)
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=dev)
+    _need(loss.dtype == torch.float32 and loss.numel() == 1, "loss must be a float32 scalar")
+    errors = []
+
+    def cut(v, r0, n):
+        return v[r0:r0 + n] if isinstance(v, torch.Tensor) and v.dim() >= 1 and v.shape[0] == N else v
+
+    def callback(ctx, row0, rows, logits_ptr, ld, v, loss_ptr, stream_ptr):
+        try:
+            strm = (torch.cuda.ExternalStream(stream_ptr, device=dev) if stream_ptr
+                    else torch.cuda.default_stream(dev))
+            with torch.cuda.stream(strm):
+                logits = torch.as_tensor(_DeviceView(logits_ptr, (rows, v), (ld * 2, 2), "<i2"),
+                                         device=dev).view(torch.bfloat16)
+                acc = torch.as_tensor(_DeviceView(loss_ptr, (1,), (4,), "<f4"), device=dev)
+                args = [cut(a, row0, rows) for a in loss_args]
+                kwargs = {k: cut(a, row0, rows) for k, a in loss_kwargs.items()}
+                chunk_loss, grad_logits = loss_and_grad_fn(logits, *args, **kwargs)
+                if tuple(grad_logits.shape) != (rows, v):
+                    raise ValueError(f"grad_logits shape {tuple(grad_logits.shape)} != {(rows, v)}")
+                logits.copy_(grad_logits)
+                acc.add_(torch.as_tensor(chunk_loss, device=dev).reshape(1).to(torch.float32))
+            return GH_OK
+        except BaseException as e:  # reported after the call returns
+            errors.append(e)
+            return GH_ERR_INVALID_ARG
+
+    fn = CHUNK_LOSS_FN(callback)
+    st = lib().gh_chunked_linear_loss(_ptr(inputs), _ptr(weight), N, D, V, int(chunk), GH_ACCUM[accum], fn, None,
+                                      _ptr(loss), _ptr(grad_inputs), _ptr(grad_weight), _stream_handle(stream))
+    if errors:
+        raise errors[0]
+    _check(st, "gh_chunked_linear_loss")
+    return loss, grad_inputs, grad_weight
+
+
+def gh_ce_vjp(logits, targets, row_loss, g, ignore_index: int = -100, *, grad=None, stream=None):
+    """Logits gradient of the per-row cross-entropy for upstream gradients ``g``
+    (one call into ``gh_ce_vjp``): ``grad[r] = g[r] * (softmax(logits[r]) - onehot(targets[r]))``.
+
+    ``row_loss`` is the forward's z-free row loss ``lse - x_t`` (``gh_ce_fwd``
+    with ``z_loss=0``), ``g`` float32 [B]; both CUDA.  ``grad`` (optional
+    output, may be ``logits`` itself) is allocated when not given.  Returns ``grad``.
+    """
+    import torch
+    _need(logits.dim() == 2 and logits.is_cuda and logits.is_contiguous(), "logits: contiguous CUDA [B, V]")
+    _need(logits.dtype in (torch.float32, torch.bfloat16), "logits dtype must be float32 or bfloat16")
+    B, V = logits.shape
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
+          and targets.shape == (B,), "targets: contiguous CUDA int64 [B]")
+    for name, v in (("row_loss", row_loss), ("g", g)):
+        _need(v.dtype == torch.float32 and v.is_cuda and v.is_contiguous() and v.shape == (B,),
+              f"{name}: contiguous CUDA float32 [B]")
+    if grad is None:
+        grad = torch.empty_like(logits)
+    _need(grad.shape == logits.shape and grad.dtype == logits.dtype and grad.is_contiguous(), "grad mismatch")
+    dtype = GH_F32 if logits.dtype == torch.float32 else GH_BF16
+    st = lib().gh_ce_vjp(_ptr(logits), _ptr(targets), B, V, dtype, int(ignore_index), _ptr(row_loss), _ptr(g),
+                         _ptr(grad), _stream_handle(stream))
+    _check(st, "gh_ce_vjp")
+    return grad
+
+
 def gh_selective_log_softmax(logits, index, *, out=None, stream=None):
     """``log_softmax(logits)[..., index]`` per row without the full log-probabilities
     (one call into ``gh_selective_log_softmax``).
@@ -276,7 +383,7 @@ def gh_linear_ce(inputs, weight, targets, ignore_index: int = -100, reduction: s
     return loss, grad_inputs, grad_weight
 
 
-GH_KERNEL = {"ce_row": 0, "logits_gemm": 1, "chunk_ce": 2, "dx_gemm": 3, "dw_gemm": 4}
+GH_KERNEL = {"ce_row": 0, "logits_gemm": 1, "chunk_ce": 2, "dx_gemm": 3, "dw_gemm": 4, "ce_vjp": 5}
 
 
 def gh_profile_enable(enable: bool = True) -> None:
@@ -304,7 +411,9 @@ def gh_get_device_status(stream=None) -> int:
 
 __all__ = [
     "GhError", "lib", "header_symbols", "status_string", "gh_status_string", "gh_version",
-    "gh_ce_fwd_bwd", "gh_ce_fwd_bwd_noalloc", "GH_NOALLOC_MAX_ROWS", "gh_linear_ce", "gh_get_device_status", "gh_profile_enable", "gh_profile_read",
+    "gh_ce_fwd_bwd", "gh_ce_fwd_bwd_noalloc", "GH_NOALLOC_MAX_ROWS", "gh_ce_fwd", "gh_selective_log_softmax",
+    "gh_ce_vjp", "gh_linear_ce", "gh_chunked_linear_loss", "CHUNK_LOSS_FN",
+    "gh_get_device_status", "gh_profile_enable", "gh_profile_read",
     "gh_launch_count", "GH_KERNEL",
     "GH_OK", "GH_ERR_INVALID_ARG", "GH_ERR_UNSUPPORTED", "GH_ERR_ALLOC", "GH_ERR_CUDA",
     "GH_ERR_TIMEOUT", "GH_ERR_TARGET_RANGE", "GH_REDUCTION", "GH_ACCUM", "GH_F32", "GH_BF16",

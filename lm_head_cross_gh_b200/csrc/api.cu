@@ -166,6 +166,26 @@ gh_status_t gh_ce_fwd(const void* logits, const int64_t* targets, int64_t B, int
   return st;
 }
 
+gh_status_t gh_ce_vjp(const void* logits, const int64_t* targets, int64_t B, int64_t V, gh_dtype_t dtype,
+                      int64_t ignore_index, const float* row_loss, const float* g, void* grad, void* stream_) {
+  if (B < 0 || V < 1 || V >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
+  if (dtype != GH_F32 && dtype != GH_BF16) return GH_ERR_INVALID_ARG;
+  if (B > 0 && (!logits || !targets || !row_loss || !g || !grad)) return GH_ERR_INVALID_ARG;
+  const int es = dtype == GH_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(logits) % es) || (reinterpret_cast<uintptr_t>(grad) % es) ||
+      (reinterpret_cast<uintptr_t>(targets) % 8) || (reinterpret_cast<uintptr_t>(row_loss) % 4) ||
+      (reinterpret_cast<uintptr_t>(g) % 4))
+    return GH_ERR_INVALID_ARG;
+  if (grad != logits && B > 0) {
+    const uintptr_t l0 = reinterpret_cast<uintptr_t>(logits), g0 = reinterpret_cast<uintptr_t>(grad);
+    const uintptr_t bytes = static_cast<uintptr_t>(B) * static_cast<uintptr_t>(V) * es;
+    if (l0 < g0 + bytes && g0 < l0 + bytes) return GH_ERR_INVALID_ARG;
+  }
+  if (B == 0) return GH_OK;
+  return ce_vjp_launch(logits, targets, row_loss, g, grad, B, V, ignore_index, dtype,
+                       static_cast<cudaStream_t>(stream_));
+}
+
 gh_status_t gh_selective_log_softmax(const void* logits, const int64_t* index, int64_t rows, int64_t V,
                                      gh_dtype_t dtype, float* out, void* stream_) {
   if (rows < 0 || V < 1 || V >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
@@ -218,6 +238,34 @@ gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* 
   a.loss = loss;
   a.dX = grad_inputs;
   a.dW = grad_weight;
+  return linear_ce_run(a, static_cast<cudaStream_t>(stream_));
+}
+
+gh_status_t gh_chunked_linear_loss(const void* inputs, const void* weight, int64_t N, int64_t D, int64_t V,
+                                   int64_t chunk, gh_accum_t accum_dtype, gh_chunk_loss_fn loss_fn, void* ctx,
+                                   float* loss, void* grad_inputs, void* grad_weight, void* stream_) {
+  if (N < 0 || D < 1 || V < 1 || V >= (int64_t(1) << 31) || D >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
+  if (D % 8) return GH_ERR_INVALID_ARG;
+  if (accum_dtype != GH_ACCUM_FP32 && accum_dtype != GH_ACCUM_WEIGHT) return GH_ERR_INVALID_ARG;
+  if (!loss_fn || !loss || !weight || !grad_weight) return GH_ERR_INVALID_ARG;
+  if (N > 0 && (!inputs || !grad_inputs)) return GH_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(inputs) % 16) || (reinterpret_cast<uintptr_t>(weight) % 16) ||
+      (reinterpret_cast<uintptr_t>(grad_inputs) % 16) || (reinterpret_cast<uintptr_t>(grad_weight) % 16) ||
+      (reinterpret_cast<uintptr_t>(loss) % 4))
+    return GH_ERR_INVALID_ARG;
+  LinearCeArgs a{};
+  a.X = inputs;
+  a.W = weight;
+  a.N = N;
+  a.D = D;
+  a.V = V;
+  a.chunk = chunk;
+  a.accum = accum_dtype;
+  a.loss = loss;
+  a.dX = grad_inputs;
+  a.dW = grad_weight;
+  a.loss_fn = loss_fn;
+  a.loss_ctx = ctx;
   return linear_ce_run(a, static_cast<cudaStream_t>(stream_));
 }
 

@@ -218,7 +218,9 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   uint16_t* dX = static_cast<uint16_t*>(a.dX);
   uint16_t* dW = static_cast<uint16_t*>(a.dW);
 
-  st = ce_count_launch(a.targets, N, V, a.ignore_index, n_valid, stream);
+  const bool custom = a.loss_fn != nullptr;
+  st = custom ? (cudaMemsetAsync(a.loss, 0, sizeof(float), stream) == cudaSuccess ? GH_OK : GH_ERR_CUDA)
+              : ce_count_launch(a.targets, N, V, a.ignore_index, n_valid, stream);
   // W as the K-major B operand of the logits GEMM and the N-major B operand of
   // dX; the weight-gradient output (bf16) and accumulator (fp32) maps.
   CUtensorMap tm_w_k, tm_w_n, tm_dw_out, tm_acc, tm_ws;
@@ -246,22 +248,28 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, GH_KERNEL_LOGITS_GEMM, stream);
     if (st != GH_OK) break;
 
-    // 2: per-row loss and the logits gradient, in place
-    CeArgs ca{};
-    ca.logits = L;
-    ca.grad = L;
-    ca.targets = a.targets + c0;
-    ca.V = V;
-    ca.ld = ld;
-    ca.ignore_index = a.ignore_index;
-    ca.z = a.z;
-    ca.mean = a.mean;
-    ca.n_valid = n_valid;
-    ca.row_loss = row_loss + c0;
-    ca.congruent = 1;
-    ca.profile_kind = GH_KERNEL_CHUNK_CE;
-    st = ce_launch(ca, rows, GH_BF16, stream);
-    if (st != GH_OK) break;
+    // 2: per-row loss and the logits gradient, in place (the caller's loss, or
+    // the cross-entropy row kernels)
+    if (custom) {
+      st = a.loss_fn(a.loss_ctx, c0, rows, L, ld, V, a.loss, stream);
+      if (st != GH_OK) break;
+    } else {
+      CeArgs ca{};
+      ca.logits = L;
+      ca.grad = L;
+      ca.targets = a.targets + c0;
+      ca.V = V;
+      ca.ld = ld;
+      ca.ignore_index = a.ignore_index;
+      ca.z = a.z;
+      ca.mean = a.mean;
+      ca.n_valid = n_valid;
+      ca.row_loss = row_loss + c0;
+      ca.congruent = 1;
+      ca.profile_kind = GH_KERNEL_CHUNK_CE;
+      st = ce_launch(ca, rows, GH_BF16, stream);
+      if (st != GH_OK) break;
+    }
 
     // 3: dX_c = G_c W (K split into fp32 partials when the tiles alone leave SMs idle)
     sm100::GemmArgs g3 = gemm_args(rows, static_cast<int>(D), static_cast<int>(V), 1, sm100::kEpiStoreBf16);
@@ -310,7 +318,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     note_launch();
     if (e != cudaSuccess) st = GH_ERR_CUDA;
   }
-  if (st == GH_OK) st = ce_reduce_launch(row_loss, N, n_valid, a.mean, a.loss, stream);
+  if (st == GH_OK && !custom) st = ce_reduce_launch(row_loss, N, n_valid, a.mean, a.loss, stream);
   scratch_free(scratch, stream);
   return st;
 }

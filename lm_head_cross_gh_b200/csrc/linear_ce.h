@@ -21,6 +21,8 @@ struct LinearCeArgs {
   float* loss;             // device scalar
   void* dX;                // [N, D] bf16
   void* dW;                // [V, D] bf16
+  gh_chunk_loss_fn loss_fn;  // null: cross-entropy; else the caller's loss per chunk
+  void* loss_ctx;
 };
 
 gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream);
