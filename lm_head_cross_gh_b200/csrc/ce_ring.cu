@@ -406,6 +406,19 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
 // skip both copies and get a zero gradient row.
 // ---------------------------------------------------------------------------
 
+// Pass 2 of a row follows pass 1 of the next row, so lse is ready when its
+// copies land and the consumers never wait on the finalizer.  For rows of
+// kLongRowBytes or more that order puts about three rows of other traffic
+// between the two copies of a piece (1.5 MB per SM for 512 KiB rows: more
+// than L2 holds across 148 SMs), so pass 2 would read HBM again; those rows
+// run pass 2 straight after their own pass 1 instead (about one row between
+// the copies), and the consumers wait for the row's lse once, while the
+// producer's pass-2 copies are already in flight.
+#ifndef GH_RING_LONG_ROW_BYTES
+#define GH_RING_LONG_ROW_BYTES (256 * 1024)
+#endif
+constexpr int64_t kLongRowBytes = GH_RING_LONG_ROW_BYTES;
+
 // Gradient of one 16-byte chunk: element e0 + j of the row gets
 // coef 2^(x_j log2e + nl) (nl = -lse log2e), minus scale at the target (chunk
 // position tj, or -1).  `dst` is the chunk's first element in the gradient row.
@@ -440,6 +453,8 @@ __device__ __forceinline__ void grad_chunk(const uint4& q, float coef, float nl,
 template <typename T>
 __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
   constexpr int ES = Elem<T>::kBytes;
+  // Long rows run pass 2 right after their own pass 1 (see kLongRowBytes).
+  const bool lag0 = a.V * ES >= kLongRowBytes;
   extern __shared__ __align__(128) uint8_t smem[];
   RingShared& sh = *reinterpret_cast<RingShared*>(smem);
   uint8_t* ring = smem + kRingHdrBytes;
@@ -502,7 +517,11 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
         const int64_t t_next = has ? target_of(row + G) : 0;
         const bool valid = has && ring_target_valid(a, t);
         if (valid && !issue_row(row)) break;
-        if (prev_valid && !issue_row(row - G)) break;
+        if (lag0) {
+          if (valid && !issue_row(row)) break;
+        } else if (prev_valid && !issue_row(row - G)) {
+          break;
+        }
         if (!has || *abort_flag) break;
         prev_valid = valid;
         t = t_next;
@@ -712,7 +731,14 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
       ++k;
       if (!ok) break;
     }
-    if (row - G >= first) {  // pass 2 (or the zero row) of the previous row
+    if (lag0) {  // pass 2 (or the zero row) of this row
+      if (valid) {
+        pass2(row, t, kr);
+        if (!ok) break;
+      } else if (has) {
+        zero_row(row);
+      }
+    } else if (row - G >= first) {  // pass 2 (or the zero row) of the previous row
       if (prev_valid) {
         pass2(row - G, prev_t, prev_k);
         if (!ok) break;
