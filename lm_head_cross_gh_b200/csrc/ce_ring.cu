@@ -413,7 +413,9 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
 // than L2 holds across 148 SMs), so pass 2 would read HBM again; those rows
 // run pass 2 straight after their own pass 1 instead (about one row between
 // the copies), and the consumers wait for the row's lse once, while the
-// producer's pass-2 copies are already in flight.
+// producer's pass-2 copies are already in flight.  Their pass-1 copies mark
+// the lines evict-last and the pass-2 copies evict-first, so the row stays in
+// L2 between the two (the gradient stores are evict-first too).
 #ifndef GH_RING_LONG_ROW_BYTES
 #define GH_RING_LONG_ROW_BYTES (256 * 1024)
 #endif
@@ -497,7 +499,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
     // ---------------- producer: pass 1 of row i, then pass 2 of row i - 1 ----------------
     if (lane == 0) {
       uint32_t n = 0;  // pieces issued
-      auto issue_row = [&](int64_t row) -> bool {
+      // long rows: pass-1 copies keep their lines in L2 for pass 2, pass-2
+      // copies let them go
+      const uint64_t pol_keep = l2_policy_evict_last(), pol_drop = l2_policy_evict_first();
+      auto issue_row = [&](int64_t row, bool first_pass) -> bool {
         const RingRow r = ring_row<ES>(a, row);
         const int np = ring_pieces(r);
         for (int p = 0; p < np; ++p, ++n) {
@@ -506,7 +511,11 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
           const int c0 = r.c_lo + p * kRingPieceChunks;
           const uint32_t bytes = 16u * static_cast<uint32_t>(tmin(kRingPieceChunks, r.c_hi - c0));
           mbar_arrive_expect_tx(&sh.full[s], bytes);
-          bulk_g2s(ring + s * kRingPieceBytes, r.base + 16 * static_cast<int64_t>(c0), bytes, &sh.full[s]);
+          if (lag0)
+            bulk_g2s_hint(ring + s * kRingPieceBytes, r.base + 16 * static_cast<int64_t>(c0), bytes, &sh.full[s],
+                          first_pass ? pol_keep : pol_drop);
+          else
+            bulk_g2s(ring + s * kRingPieceBytes, r.base + 16 * static_cast<int64_t>(c0), bytes, &sh.full[s]);
         }
         return true;
       };
@@ -516,10 +525,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
         const bool has = row < a.B;
         const int64_t t_next = has ? target_of(row + G) : 0;
         const bool valid = has && ring_target_valid(a, t);
-        if (valid && !issue_row(row)) break;
+        if (valid && !issue_row(row, true)) break;
         if (lag0) {
-          if (valid && !issue_row(row)) break;
-        } else if (prev_valid && !issue_row(row - G)) {
+          if (valid && !issue_row(row, false)) break;
+        } else if (prev_valid && !issue_row(row - G, false)) {
           break;
         }
         if (!has || *abort_flag) break;
