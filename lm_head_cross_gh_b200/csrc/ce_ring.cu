@@ -409,15 +409,17 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
 // Pass 2 of a row follows pass 1 of the next row, so lse is ready when its
 // copies land and the consumers never wait on the finalizer.  For rows of
 // kLongRowBytes or more that order puts about three rows of other traffic
-// between the two copies of a piece (1.5 MB per SM for 512 KiB rows: more
-// than L2 holds across 148 SMs), so pass 2 would read HBM again; those rows
+// between the two copies of a piece (3 x 148 x 128 KiB = 57 MB and up, 227 MB
+// for 512 KiB rows: too much for L2 next to the gradient stores), so pass 2
+// would read HBM again (measured: 112 KiB rows run at 82% of the copy rate
+// in this order, 128 KiB rows at 72%); those rows
 // run pass 2 straight after their own pass 1 instead (about one row between
 // the copies), and the consumers wait for the row's lse once, while the
 // producer's pass-2 copies are already in flight.  Their pass-1 copies mark
 // the lines evict-last and the pass-2 copies evict-first, so the row stays in
 // L2 between the two (the gradient stores are evict-first too).
 #ifndef GH_RING_LONG_ROW_BYTES
-#define GH_RING_LONG_ROW_BYTES (256 * 1024)
+#define GH_RING_LONG_ROW_BYTES (120 * 1024)
 #endif
 constexpr int64_t kLongRowBytes = GH_RING_LONG_ROW_BYTES;
 
