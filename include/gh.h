@@ -41,8 +41,8 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Work is enqueued on it and the call returns without waiting;
  *    outputs are valid once the stream reaches that point.  The library
- *    allocates its scratch stream-ordered (cudaMallocAsync/cudaFreeAsync) on
- *    the same stream.
+ *    allocates its scratch stream-ordered on the same stream, from a memory
+ *    pool it keeps per device (freed memory is kept for later calls).
  *  - Arguments are validated on the host before anything is enqueued:
  *    null pointers, negative sizes, unknown enums and non-finite z give
  *    GH_ERR_INVALID_ARG and nothing runs.  B == 0 (or N == 0) writes loss = 0.
@@ -109,11 +109,12 @@ gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B,
 
 /*
  * gh_ce_fwd_bwd_noalloc — gh_ce_fwd_bwd for callers that cannot allocate.
- * The pages have no counterpart; this entry point exists for callers whose
- * device memory is already owned in full by another allocator (a framework's
- * caching allocator, or a fixed arena planned ahead of time), where the
- * cudaMallocAsync that gh_ce_fwd_bwd makes for its scratch could fail in the
- * middle of a step, and for loops that forbid allocator calls inside a step.
+ * The Greyhound API has no counterpart; this entry point exists for callers
+ * whose device memory is already owned in full by another allocator (a
+ * framework's caching allocator, or a fixed arena planned ahead of time),
+ * where the stream-ordered allocation gh_ce_fwd_bwd makes for its scratch
+ * could fail in the middle of a step, and for loops that forbid allocator
+ * calls inside a step.
  *
  * Arguments, results and errors are those of gh_ce_fwd_bwd, except:
  *  - B is limited to 65536 rows: the scratch is a fixed array of

@@ -22,7 +22,8 @@ Sources (the Greyhound functional API page, ``greyhound.nn.functional``):
 * nuvec ``FastOp::CrossEntropy`` / ``CrossEntropyVjp`` — the row loss
   definition and its logits gradient.
 
-Readings where the pages are silent (each is listed in the design notes):
+Readings where the API documentation is silent (each is listed in the design
+notes):
 z-loss is ``z * lse**2`` per valid token, added before the reduction; ``mean``
 with no valid token returns 0 with zero gradients; ``mean`` across chunks
 divides by the global valid-token count; a target equal to ``ignore_index`` is
@@ -30,7 +31,8 @@ ignored even when it lies in [0, V); other targets outside [0, V) are an error.
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against closed
 forms, invariants, finite differences, a materialised brute force and
-``torch.nn.functional.cross_entropy`` (the library routine the pages name).
+``torch.nn.functional.cross_entropy`` (the PyTorch routine the z-free,
+unchunked case reduces to).
 """
 from .ce import (bf16_round, cross_entropy, ce_rows, n_valid_and_scale,
                  selective_log_softmax)
