@@ -454,11 +454,13 @@ __device__ __forceinline__ void grad_chunk(const uint4& q, float coef, float nl,
   }
 }
 
-template <typename T>
+// LONG: rows of kLongRowBytes or more (pass 2 right after the row's own pass 1,
+// cache-hinted copies).  The order is a template parameter so that each
+// instantiation inlines the two passes once (the instruction cache is small).
+template <typename T, bool LONG>
 __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
   constexpr int ES = Elem<T>::kBytes;
-  // Long rows run pass 2 right after their own pass 1 (see kLongRowBytes).
-  const bool lag0 = a.V * ES >= kLongRowBytes;
+  constexpr bool lag0 = LONG;
   extern __shared__ __align__(128) uint8_t smem[];
   RingShared& sh = *reinterpret_cast<RingShared*>(smem);
   uint8_t* ring = smem + kRingHdrBytes;
@@ -513,7 +515,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
           const int c0 = r.c_lo + p * kRingPieceChunks;
           const uint32_t bytes = 16u * static_cast<uint32_t>(tmin(kRingPieceChunks, r.c_hi - c0));
           mbar_arrive_expect_tx(&sh.full[s], bytes);
-          if (lag0)
+          if constexpr (lag0)
             bulk_g2s_hint(ring + s * kRingPieceBytes, r.base + 16 * static_cast<int64_t>(c0), bytes, &sh.full[s],
                           first_pass ? pol_keep : pol_drop);
           else
@@ -528,7 +530,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
         const int64_t t_next = has ? target_of(row + G) : 0;
         const bool valid = has && ring_target_valid(a, t);
         if (valid && !issue_row(row, true)) break;
-        if (lag0) {
+        if constexpr (lag0) {
           if (valid && !issue_row(row, false)) break;
         } else if (prev_valid && !issue_row(row - G, false)) {
           break;
@@ -742,7 +744,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
       ++k;
       if (!ok) break;
     }
-    if (lag0) {  // pass 2 (or the zero row) of this row
+    if constexpr (lag0) {  // pass 2 (or the zero row) of this row
       if (valid) {
         pass2(row, t, kr);
         if (!ok) break;
@@ -781,12 +783,18 @@ RingKernel ring_kernel_for(int es, int mode) {
 int ce_ring_smem_bytes() { return kRingHdrBytes + kRingSlots * kRingPieceBytes; }
 
 gh_status_t ce_ring_launch(const CeArgs& a, int es, int grid, cudaStream_t stream) {
-  const RingKernel kern = a.mode == kModeFwdBwd ? (es == 4 ? ce_ring2_kernel<float> : ce_ring2_kernel<uint16_t>)
-                                                : ring_kernel_for(es, a.mode);
-  static bool raised[64][2][3] = {};
+  const bool long_rows = a.V * es >= kLongRowBytes;
+  RingKernel kern;
+  if (a.mode == kModeFwdBwd) {
+    if (es == 4) kern = long_rows ? ce_ring2_kernel<float, true> : ce_ring2_kernel<float, false>;
+    else kern = long_rows ? ce_ring2_kernel<uint16_t, true> : ce_ring2_kernel<uint16_t, false>;
+  } else {
+    kern = ring_kernel_for(es, a.mode);
+  }
+  static bool raised[64][2][4] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GH_ERR_CUDA;
-  const int kv = es == 4, km = a.mode;
+  const int kv = es == 4, km = a.mode == kModeFwdBwd && long_rows ? 3 : a.mode;
   if (dev < 64 && !raised[dev][kv][km]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, ce_ring_smem_bytes()) !=
         cudaSuccess)
