@@ -1,10 +1,10 @@
-// Forward-only cross-entropy rows (the loss without its gradient, and the
-// selective log-softmax x[index] - lse) as one streaming pipeline per SM.
+// Cross-entropy rows as one streaming pipeline per SM: the forward-only kernel
+// (the loss without its gradient, and the selective log-softmax x[index] -
+// lse) and, further down, the two-pass forward+backward kernel built on it.
 //
-// Without a gradient pass nothing has to stay in shared memory once it has
-// been read, so the row-buffer design of the forward+backward kernel (a whole
-// row resident, the next row's copy waiting for the buffer) gives way to a ring
-// of fixed-size pieces that runs across row boundaries:
+// Nothing has to stay in shared memory once it has been read, so instead of
+// a whole row resident in shared memory (the row kernel in ce.cu) a ring of
+// fixed-size pieces runs across row boundaries:
 //
 //   warp 16 (producer)   walks this CTA's rows and their pieces in order and
 //                        starts a bulk copy into the next free ring slot;
@@ -397,13 +397,14 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
 // Pass 1 of row k is the forward kernel's (online max / sum, the finalizer
 // merges, writes the row loss and publishes lse); pass 2 of row k copies the
 // row into the ring again and stores the gradient scale (1 + 2 z lse) exp(x -
-// lse), less scale at the target, straight from registers to global.  The
-// producer interleaves the passes one row apart -- pass 1 of row k, then pass 2
-// of row k - 1 -- so lse(k - 1) is ready when its pass 2 lands and the row was
-// read from HBM one row earlier: the second copy comes from L2 (126 MB; all
-// SMs together keep about two rows each in flight).  HBM sees one read and one
-// write of every logit; every element costs two exponentials.  Ignored rows
-// skip both copies and get a zero gradient row.
+// lse), less scale at the target, straight from registers to global.  For
+// rows shorter than kLongRowBytes the producer interleaves the passes one row
+// apart -- pass 1 of row k, then pass 2 of row k - 1 -- so lse(k - 1) is ready
+// when its pass 2 lands and the row was read from HBM one row earlier: the
+// second copy comes from L2.  Longer rows run pass 2 straight after their own
+// pass 1, with L2 eviction hints (below).  HBM sees one read and one write of
+// every logit; every element costs two exponentials.  Ignored rows skip both
+// copies and get a zero gradient row.
 // ---------------------------------------------------------------------------
 
 // Pass 2 of a row follows pass 1 of the next row, so lse is ready when its
