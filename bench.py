@@ -51,11 +51,37 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_text(src: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace collapsed, so a
+    comment-only edit keeps the digest of the code it describes."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == '"' or c == "'":  # string or char literal, copied whole
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_digest(files):
+    """sha1 (12 hex digits) of the code of `files`, comments and layout aside."""
     h = hashlib.sha1()
     for f in files:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(code_text(fh.read()).encode())
     return h.hexdigest()[:12]
 
 
