@@ -1,0 +1,131 @@
+"""Greyhound-style functional API (the names and signatures of
+``greyhound.nn.functional``) over the C ABI, with PyTorch autograd.
+
+Every loss is computed by the library's kernels in the forward call, together
+with its gradients (they come out of the same passes); ``backward`` returns
+them, scaled by the upstream gradient when that is not 1.  PyTorch only holds
+the tensors: there is no other implementation behind these functions.
+
+* ``cross_entropy(logits, target, ignore_index, reduction, z_loss_multiplier)``
+* ``chunked_linear_cross_entropy(inputs, weight, target, ignore_index, reduction,
+  z_loss_multiplier, grad_weight_accum_dtype)``
+* ``chunked_linear_loss(inputs, weight, loss_and_grad_fn, *loss_args, chunk_size,
+  grad_weight_accum_dtype, **loss_kwargs)``
+* ``autograd_loss_and_logits_grad(loss_fn)``: adapts a PyTorch scalar loss to
+  the ``(loss, grad_logits)`` contract of ``chunked_linear_loss``
+* ``selective_log_softmax(logits, index)`` (forward only)
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (gh_ce_fwd, gh_ce_fwd_bwd, gh_chunked_linear_loss, gh_linear_ce, gh_selective_log_softmax)
+
+__all__ = ["cross_entropy", "chunked_linear_cross_entropy", "chunked_linear_loss",
+           "autograd_loss_and_logits_grad", "selective_log_softmax"]
+
+
+def _scaled(grad, g):
+    """grad * g for a scalar upstream gradient g, without a pass when g == 1."""
+    if grad is None:
+        return None
+    if g.numel() == 1 and bool(g.reshape(()) == 1):
+        return grad
+    return grad * g.to(grad.dtype)
+
+
+class _CrossEntropy(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, logits, target, ignore_index, reduction, z):
+        V = logits.shape[-1]
+        x = logits.reshape(-1, V).contiguous()
+        t = target.reshape(-1).contiguous()
+        ctx.shape = logits.shape
+        if ctx.needs_input_grad[0]:
+            loss, grad = gh_ce_fwd_bwd(x, t, ignore_index, reduction, z)
+            ctx.save_for_backward(grad)
+        else:
+            loss, _ = gh_ce_fwd(x, t, ignore_index, reduction, z)
+        return loss
+
+    @staticmethod
+    def backward(ctx, g):
+        (grad,) = ctx.saved_tensors
+        return _scaled(grad, g).view(ctx.shape), None, None, None, None
+
+
+def cross_entropy(logits, target, ignore_index: int = -100, reduction: str = "mean",
+                  z_loss_multiplier: float = 0.0):
+    """Cross-entropy of ``logits`` [..., V] (float32 or bfloat16, CUDA) against
+    ``target`` [...] (int64) with ``ignore_index``, ``"mean"``/``"sum"`` reduction
+    and the z-loss ``z_loss_multiplier * lse**2``.  Returns a float32 scalar; its
+    backward gives the logits gradient computed in the forward pass."""
+    return _CrossEntropy.apply(logits, target, ignore_index, reduction, float(z_loss_multiplier))
+
+
+class _LinearCE(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, inputs, weight, target, ignore_index, reduction, z, accum):
+        loss, dX, dW = gh_linear_ce(inputs.contiguous(), weight.contiguous(), target.contiguous(), ignore_index,
+                                    reduction, z, 0, accum)
+        ctx.save_for_backward(dX, dW)
+        return loss
+
+    @staticmethod
+    def backward(ctx, g):
+        dX, dW = ctx.saved_tensors
+        return (_scaled(dX, g) if ctx.needs_input_grad[0] else None,
+                _scaled(dW, g) if ctx.needs_input_grad[1] else None, None, None, None, None, None)
+
+
+def chunked_linear_cross_entropy(inputs, weight, target, ignore_index: int = -100, reduction: str = "mean",
+                                 z_loss_multiplier: float = 0.0, grad_weight_accum_dtype: str = "fp32"):
+    """Cross-entropy of ``inputs @ weight.T`` (bf16 [BT, D] and [V, D], CUDA)
+    computed in row chunks without materialising the logits; the backward gives
+    grad_inputs and grad_weight (accumulated in fp32 or in the weight dtype)."""
+    return _LinearCE.apply(inputs, weight, target, ignore_index, reduction, float(z_loss_multiplier),
+                           grad_weight_accum_dtype)
+
+
+class _ChunkedLoss(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, inputs, weight, loss_and_grad_fn, chunk, accum, args, kwargs):
+        loss, dX, dW = gh_chunked_linear_loss(inputs.contiguous(), weight.contiguous(), loss_and_grad_fn, *args,
+                                              chunk=chunk, accum=accum, **kwargs)
+        ctx.save_for_backward(dX, dW)
+        return loss
+
+    @staticmethod
+    def backward(ctx, g):
+        dX, dW = ctx.saved_tensors
+        return (_scaled(dX, g) if ctx.needs_input_grad[0] else None,
+                _scaled(dW, g) if ctx.needs_input_grad[1] else None, None, None, None, None, None)
+
+
+def chunked_linear_loss(inputs, weight, loss_and_grad_fn, *loss_args, chunk_size=None,
+                        grad_weight_accum_dtype: str = "fp32", **loss_kwargs):
+    """``inputs @ weight.T`` in row chunks followed by the caller's
+    ``loss_and_grad_fn(logits_chunk, *chunk_args, **chunk_kwargs) -> (loss,
+    grad_logits)``; tensor arguments whose leading dimension is BT are sliced to
+    the chunk's rows.  Returns the sum of the chunk losses."""
+    return _ChunkedLoss.apply(inputs, weight, loss_and_grad_fn, int(chunk_size or 0), grad_weight_accum_dtype,
+                              loss_args, loss_kwargs)
+
+
+def autograd_loss_and_logits_grad(loss_fn):
+    """Adapt a PyTorch scalar loss ``loss_fn(logits, *args, **kwargs)`` to the
+    ``(loss, grad_logits)`` contract: the loss is evaluated on an fp32 copy of
+    the chunk logits and differentiated by autograd; the gradient comes back in
+    the logits dtype."""
+    def loss_and_grad(logits, *args, **kwargs):
+        with torch.enable_grad():
+            x = logits.detach().float().requires_grad_(True)
+            loss = loss_fn(x, *args, **kwargs)
+            (g,) = torch.autograd.grad(loss, x)
+        return loss.detach(), g.to(logits.dtype)
+    return loss_and_grad
+
+
+def selective_log_softmax(logits, index):
+    """``log_softmax(logits)`` gathered at ``index`` (forward only): float32 [...]."""
+    return gh_selective_log_softmax(logits.contiguous(), index.contiguous())
