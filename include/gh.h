@@ -134,6 +134,30 @@ gh_status_t gh_ce_fwd_bwd_noalloc(const void* logits, const int64_t* targets, in
                                   float z_mult, float* loss, void* grad, void* stream);
 
 /*
+ * Data-parallel shards.  A batch split over ranks has one mean: every shard
+ * divides by the valid count of the whole batch.  gh_count_valid writes a
+ * shard's count; the caller sums the counts over the ranks (one all-reduce of
+ * an int64) and passes the total to the _shard entry points, which are
+ * gh_ce_fwd_bwd / gh_linear_ce with that count in place of their own.  Their
+ * losses and gradients are then the shard's terms of the batch's: the loss is
+ * all-reduced (sum), grad_weight too; logits and input gradients are final.
+ *
+ * gh_count_valid: count = #{targets != ignore_index} over targets[0..N)
+ * (int64 device scalar, written); targets outside [0, V) that are not
+ * ignore_index record GH_ERR_TARGET_RANGE and are not counted.
+ * n_valid_total: device int64 scalar, read by the kernels (8-byte aligned).
+ */
+gh_status_t gh_count_valid(const int64_t* targets, int64_t N, int64_t V, int64_t ignore_index, int64_t* count,
+                           void* stream);
+gh_status_t gh_ce_fwd_bwd_shard(const void* logits, const int64_t* targets, int64_t B, int64_t V,
+                                gh_dtype_t dtype, int64_t ignore_index, gh_reduction_t reduction, float z_mult,
+                                const int64_t* n_valid_total, float* loss, void* grad, void* stream);
+gh_status_t gh_linear_ce_shard(const void* inputs, const void* weight, const int64_t* targets, int64_t N,
+                               int64_t D, int64_t V, int64_t chunk, gh_accum_t accum_dtype, int64_t ignore_index,
+                               gh_reduction_t reduction, float z_mult, const int64_t* n_valid_total, float* loss,
+                               void* grad_inputs, void* grad_weight, void* stream);
+
+/*
  * gh_ce_fwd — the cross-entropy loss of gh_ce_fwd_bwd without its gradient:
  * the evaluation form (a forward with no tape and no gradients), reading the
  * logits once.

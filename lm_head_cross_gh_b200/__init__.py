@@ -67,6 +67,14 @@ def lib() -> ctypes.CDLL:
     L.gh_ce_fwd_bwd.restype = c_int
     L.gh_ce_fwd_bwd_noalloc.argtypes = list(L.gh_ce_fwd_bwd.argtypes)
     L.gh_ce_fwd_bwd_noalloc.restype = c_int
+    L.gh_count_valid.argtypes = [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p]
+    L.gh_count_valid.restype = c_int
+    L.gh_ce_fwd_bwd_shard.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_int, c_float,
+                                      c_void_p, c_void_p, c_void_p, c_void_p]
+    L.gh_ce_fwd_bwd_shard.restype = c_int
+    L.gh_linear_ce_shard.argtypes = [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int,
+                                     c_int64, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
+    L.gh_linear_ce_shard.restype = c_int
     L.gh_ce_fwd.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_int, c_float,
                             c_void_p, c_void_p, c_void_p]
     L.gh_ce_fwd.restype = c_int
@@ -198,6 +206,70 @@ def gh_ce_fwd_bwd_noalloc(logits, targets, ignore_index: int = -100, reduction: 
                                      _stream_handle(stream))
     _check(st, "gh_ce_fwd_bwd_noalloc")
     return loss, grad
+
+
+def gh_count_valid(targets, V: int, ignore_index: int = -100, *, count=None, stream=None):
+    """Number of targets that are not ``ignore_index`` (CUDA int64 scalar tensor)."""
+    import torch
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous(), "targets: CUDA int64")
+    if count is None:
+        count = torch.empty((), dtype=torch.int64, device=targets.device)
+    _need(count.dtype == torch.int64 and count.numel() == 1 and count.is_cuda, "count: CUDA int64 scalar")
+    _check(lib().gh_count_valid(_ptr(targets), targets.numel(), int(V), int(ignore_index), _ptr(count),
+                                _stream_handle(stream)), "gh_count_valid")
+    return count
+
+
+def gh_ce_fwd_bwd_shard(logits, targets, n_valid_total, ignore_index: int = -100, reduction: str = "mean",
+                        z_loss: float = 0.0, *, grad=None, loss=None, stream=None):
+    """``gh_ce_fwd_bwd`` for one shard of a data-parallel batch: the mean divides
+    by ``n_valid_total`` (CUDA int64 scalar: the valid count of all shards)."""
+    import torch
+    _need(logits.dim() == 2 and logits.is_cuda and logits.is_contiguous(), "logits: contiguous CUDA [B, V]")
+    _need(logits.dtype in (torch.float32, torch.bfloat16), "logits dtype must be float32 or bfloat16")
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
+          and targets.shape == (logits.shape[0],), "targets: contiguous CUDA int64 [B]")
+    _need(n_valid_total.dtype == torch.int64 and n_valid_total.numel() == 1 and n_valid_total.is_cuda,
+          "n_valid_total: CUDA int64 scalar")
+    _need(reduction in GH_REDUCTION, "reduction must be 'mean' or 'sum'")
+    if grad is None:
+        grad = torch.empty_like(logits)
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=logits.device)
+    B, V = logits.shape
+    dtype = GH_F32 if logits.dtype == torch.float32 else GH_BF16
+    st = lib().gh_ce_fwd_bwd_shard(_ptr(logits), _ptr(targets), B, V, dtype, int(ignore_index),
+                                   GH_REDUCTION[reduction], float(z_loss), _ptr(n_valid_total), _ptr(loss),
+                                   _ptr(grad), _stream_handle(stream))
+    _check(st, "gh_ce_fwd_bwd_shard")
+    return loss, grad
+
+
+def gh_linear_ce_shard(inputs, weight, targets, n_valid_total, ignore_index: int = -100, reduction: str = "mean",
+                       z_loss: float = 0.0, chunk: int = 0, accum: str = "fp32", *, grad_inputs=None,
+                       grad_weight=None, loss=None, stream=None):
+    """``gh_linear_ce`` for one shard of a data-parallel batch (mean over
+    ``n_valid_total``, a CUDA int64 scalar)."""
+    import torch
+    _need(inputs.dim() == 2 and weight.dim() == 2 and inputs.shape[1] == weight.shape[1], "shapes")
+    _need(inputs.dtype == torch.bfloat16 and weight.dtype == torch.bfloat16, "inputs/weight must be bfloat16")
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
+          and targets.shape == (inputs.shape[0],), "targets: contiguous CUDA int64 [N]")
+    _need(n_valid_total.dtype == torch.int64 and n_valid_total.numel() == 1 and n_valid_total.is_cuda,
+          "n_valid_total: CUDA int64 scalar")
+    N, D = inputs.shape
+    V = weight.shape[0]
+    if grad_inputs is None:
+        grad_inputs = torch.empty_like(inputs)
+    if grad_weight is None:
+        grad_weight = torch.empty_like(weight)
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=inputs.device)
+    st = lib().gh_linear_ce_shard(_ptr(inputs), _ptr(weight), _ptr(targets), N, D, V, int(chunk), GH_ACCUM[accum],
+                                  int(ignore_index), GH_REDUCTION[reduction], float(z_loss), _ptr(n_valid_total),
+                                  _ptr(loss), _ptr(grad_inputs), _ptr(grad_weight), _stream_handle(stream))
+    _check(st, "gh_linear_ce_shard")
+    return loss, grad_inputs, grad_weight
 
 
 def gh_ce_fwd(logits, targets, ignore_index: int = -100, reduction: str = "mean", z_loss: float = 0.0, *,
@@ -413,6 +485,7 @@ __all__ = [
     "GhError", "lib", "header_symbols", "status_string", "gh_status_string", "gh_version",
     "gh_ce_fwd_bwd", "gh_ce_fwd_bwd_noalloc", "GH_NOALLOC_MAX_ROWS", "gh_ce_fwd", "gh_selective_log_softmax",
     "gh_ce_vjp", "gh_linear_ce", "gh_chunked_linear_loss", "CHUNK_LOSS_FN",
+    "gh_count_valid", "gh_ce_fwd_bwd_shard", "gh_linear_ce_shard",
     "gh_get_device_status", "gh_profile_enable", "gh_profile_read",
     "gh_launch_count", "GH_KERNEL",
     "GH_OK", "GH_ERR_INVALID_ARG", "GH_ERR_UNSUPPORTED", "GH_ERR_ALLOC", "GH_ERR_CUDA",

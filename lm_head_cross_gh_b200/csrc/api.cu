@@ -71,9 +71,11 @@ using namespace gh;
 
 extern "C" {
 
-gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B, int64_t V, gh_dtype_t dtype,
-                          int64_t ignore_index, gh_reduction_t reduction, float z_mult, float* loss, void* grad,
-                          void* stream_) {
+// gh_ce_fwd_bwd and its data-parallel shard form: n_total (device) is the valid
+// count of the whole batch, or null to count this call's targets.
+static gh_status_t ce_fwd_bwd_impl(const void* logits, const int64_t* targets, int64_t B, int64_t V,
+                                   gh_dtype_t dtype, int64_t ignore_index, gh_reduction_t reduction, float z_mult,
+                                   const int64_t* n_total, float* loss, void* grad, void* stream_) {
   if (B < 0 || V < 1 || V >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
   if (dtype != GH_F32 && dtype != GH_BF16) return GH_ERR_INVALID_ARG;
   if (reduction != GH_REDUCTION_MEAN && reduction != GH_REDUCTION_SUM) return GH_ERR_INVALID_ARG;
@@ -96,11 +98,12 @@ gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B,
   void* scratch = nullptr;
   gh_status_t st = scratch_alloc(&scratch, 16 + static_cast<size_t>(B) * sizeof(float), stream);
   if (st != GH_OK) return st;
-  unsigned long long* n_valid = static_cast<unsigned long long*>(scratch);
+  unsigned long long* counter = static_cast<unsigned long long*>(scratch);
   float* row_loss = reinterpret_cast<float*>(static_cast<char*>(scratch) + 16);
+  const unsigned long long* n_valid = n_total ? reinterpret_cast<const unsigned long long*>(n_total) : counter;
 
   const int mean = reduction == GH_REDUCTION_MEAN;
-  st = ce_count_launch(targets, B, V, ignore_index, n_valid, stream);
+  st = n_total ? GH_OK : ce_count_launch(targets, B, V, ignore_index, counter, stream);
   if (st == GH_OK) {
     CeArgs a{};
     a.logits = logits;
@@ -119,6 +122,29 @@ gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B,
   if (st == GH_OK) st = ce_reduce_launch(row_loss, B, n_valid, mean, loss, stream);
   scratch_free(scratch, stream);
   return st;
+}
+
+gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B, int64_t V, gh_dtype_t dtype,
+                          int64_t ignore_index, gh_reduction_t reduction, float z_mult, float* loss, void* grad,
+                          void* stream) {
+  return ce_fwd_bwd_impl(logits, targets, B, V, dtype, ignore_index, reduction, z_mult, nullptr, loss, grad, stream);
+}
+
+gh_status_t gh_ce_fwd_bwd_shard(const void* logits, const int64_t* targets, int64_t B, int64_t V, gh_dtype_t dtype,
+                                int64_t ignore_index, gh_reduction_t reduction, float z_mult,
+                                const int64_t* n_valid_total, float* loss, void* grad, void* stream) {
+  if (!n_valid_total || (reinterpret_cast<uintptr_t>(n_valid_total) % 8)) return GH_ERR_INVALID_ARG;
+  return ce_fwd_bwd_impl(logits, targets, B, V, dtype, ignore_index, reduction, z_mult, n_valid_total, loss, grad,
+                         stream);
+}
+
+gh_status_t gh_count_valid(const int64_t* targets, int64_t N, int64_t V, int64_t ignore_index, int64_t* count,
+                           void* stream_) {
+  if (N < 0 || V < 1 || !count || (reinterpret_cast<uintptr_t>(count) % 8)) return GH_ERR_INVALID_ARG;
+  if (N > 0 && (!targets || (reinterpret_cast<uintptr_t>(targets) % 8))) return GH_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (N == 0) return cudaMemsetAsync(count, 0, sizeof(int64_t), stream) == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+  return ce_count_launch(targets, N, V, ignore_index, reinterpret_cast<unsigned long long*>(count), stream);
 }
 
 gh_status_t gh_ce_fwd(const void* logits, const int64_t* targets, int64_t B, int64_t V, gh_dtype_t dtype,
@@ -208,10 +234,10 @@ gh_status_t gh_selective_log_softmax(const void* logits, const int64_t* index, i
   return ce_launch(a, rows, dtype, static_cast<cudaStream_t>(stream_));
 }
 
-gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* targets, int64_t N, int64_t D,
-                         int64_t V, int64_t chunk, gh_accum_t accum_dtype, int64_t ignore_index,
-                         gh_reduction_t reduction, float z_mult, float* loss, void* grad_inputs, void* grad_weight,
-                         void* stream_) {
+static gh_status_t linear_ce_impl(const void* inputs, const void* weight, const int64_t* targets, int64_t N,
+                                  int64_t D, int64_t V, int64_t chunk, gh_accum_t accum_dtype, int64_t ignore_index,
+                                  gh_reduction_t reduction, float z_mult, const int64_t* n_total, float* loss,
+                                  void* grad_inputs, void* grad_weight, void* stream_) {
   if (N < 0 || D < 1 || V < 1 || V >= (int64_t(1) << 31) || D >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
   if (D % 8) return GH_ERR_INVALID_ARG;
   if (accum_dtype != GH_ACCUM_FP32 && accum_dtype != GH_ACCUM_WEIGHT) return GH_ERR_INVALID_ARG;
@@ -238,7 +264,25 @@ gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* 
   a.loss = loss;
   a.dX = grad_inputs;
   a.dW = grad_weight;
+  a.n_total = reinterpret_cast<const unsigned long long*>(n_total);
   return linear_ce_run(a, static_cast<cudaStream_t>(stream_));
+}
+
+gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* targets, int64_t N, int64_t D,
+                         int64_t V, int64_t chunk, gh_accum_t accum_dtype, int64_t ignore_index,
+                         gh_reduction_t reduction, float z_mult, float* loss, void* grad_inputs, void* grad_weight,
+                         void* stream) {
+  return linear_ce_impl(inputs, weight, targets, N, D, V, chunk, accum_dtype, ignore_index, reduction, z_mult,
+                        nullptr, loss, grad_inputs, grad_weight, stream);
+}
+
+gh_status_t gh_linear_ce_shard(const void* inputs, const void* weight, const int64_t* targets, int64_t N, int64_t D,
+                               int64_t V, int64_t chunk, gh_accum_t accum_dtype, int64_t ignore_index,
+                               gh_reduction_t reduction, float z_mult, const int64_t* n_valid_total, float* loss,
+                               void* grad_inputs, void* grad_weight, void* stream) {
+  if (!n_valid_total || (reinterpret_cast<uintptr_t>(n_valid_total) % 8)) return GH_ERR_INVALID_ARG;
+  return linear_ce_impl(inputs, weight, targets, N, D, V, chunk, accum_dtype, ignore_index, reduction, z_mult,
+                        n_valid_total, loss, grad_inputs, grad_weight, stream);
 }
 
 gh_status_t gh_chunked_linear_loss(const void* inputs, const void* weight, int64_t N, int64_t D, int64_t V,

@@ -207,7 +207,8 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   gh_status_t st = scratch_alloc(&scratch, total, stream);
   if (st != GH_OK) return st;
   char* base = static_cast<char*>(scratch);
-  unsigned long long* n_valid = reinterpret_cast<unsigned long long*>(base);
+  unsigned long long* counter = reinterpret_cast<unsigned long long*>(base);
+  const unsigned long long* n_valid = a.n_total ? a.n_total : counter;
   float* row_loss = reinterpret_cast<float*>(base + off_rows);
   uint16_t* L = reinterpret_cast<uint16_t*>(base + off_buf);
   float* acc = acc32 ? reinterpret_cast<float*>(base + off_acc) : nullptr;
@@ -219,8 +220,9 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   uint16_t* dW = static_cast<uint16_t*>(a.dW);
 
   const bool custom = a.loss_fn != nullptr;
-  st = custom ? (cudaMemsetAsync(a.loss, 0, sizeof(float), stream) == cudaSuccess ? GH_OK : GH_ERR_CUDA)
-              : ce_count_launch(a.targets, N, V, a.ignore_index, n_valid, stream);
+  st = custom    ? (cudaMemsetAsync(a.loss, 0, sizeof(float), stream) == cudaSuccess ? GH_OK : GH_ERR_CUDA)
+       : a.n_total ? GH_OK
+                   : ce_count_launch(a.targets, N, V, a.ignore_index, counter, stream);
   // W as the K-major B operand of the logits GEMM and the N-major B operand of
   // dX; the weight-gradient output (bf16) and accumulator (fp32) maps.
   CUtensorMap tm_w_k, tm_w_n, tm_dw_out, tm_acc, tm_ws;

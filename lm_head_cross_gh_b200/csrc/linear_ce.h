@@ -23,6 +23,7 @@ struct LinearCeArgs {
   void* dW;                // [V, D] bf16
   gh_chunk_loss_fn loss_fn;  // null: cross-entropy; else the caller's loss per chunk
   void* loss_ctx;
+  const unsigned long long* n_total;  // non-null: the mean divides by this count (all shards)
 };
 
 gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream);

@@ -14,6 +14,15 @@ the tensors: there is no other implementation behind these functions.
 * ``autograd_loss_and_logits_grad(loss_fn)``: adapts a PyTorch scalar loss to
   the ``(loss, grad_logits)`` contract of ``chunked_linear_loss``
 * ``selective_log_softmax(logits, index)`` (forward only)
+
+Data parallel (one process per GPU, a batch split over the ranks of a
+``torch.distributed`` group):
+
+* ``data_parallel_cross_entropy`` and ``data_parallel_chunked_linear_cross_entropy``
+  return the whole batch's loss on every rank and, in backward, this rank's share
+  of its gradients: the valid-token counts are summed over the ranks first (one
+  int64 all-reduce), every shard divides by that total, the shards' losses are
+  summed (one scalar all-reduce) and so are the weight gradients.
 """
 from __future__ import annotations
 
@@ -21,8 +30,11 @@ import torch
 
 from . import (gh_ce_fwd, gh_ce_fwd_bwd, gh_chunked_linear_loss, gh_linear_ce, gh_selective_log_softmax)
 
+_PKG = __name__.rpartition(".")[0]
+
 __all__ = ["cross_entropy", "chunked_linear_cross_entropy", "chunked_linear_loss",
-           "autograd_loss_and_logits_grad", "selective_log_softmax"]
+           "autograd_loss_and_logits_grad", "selective_log_softmax", "data_parallel_cross_entropy",
+           "data_parallel_chunked_linear_cross_entropy"]
 
 
 def _scaled(grad, g):
@@ -129,3 +141,74 @@ def autograd_loss_and_logits_grad(loss_fn):
 def selective_log_softmax(logits, index):
     """``log_softmax(logits)`` gathered at ``index`` (forward only): float32 [...]."""
     return gh_selective_log_softmax(logits.contiguous(), index.contiguous())
+
+
+def _ops(ops):
+    """The library's entry points (``ops`` stands in for them in host-only tests
+    of the collective steps)."""
+    if ops is not None:
+        return ops
+    import importlib
+    return importlib.import_module(_PKG)
+
+
+def _all_reduce_sum(t, group):
+    import torch.distributed as dist
+    dist.all_reduce(t.view(-1), op=dist.ReduceOp.SUM, group=group)
+    return t
+
+
+class _DPCrossEntropy(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, logits, target, ignore_index, reduction, z, group, ops):
+        V = logits.shape[-1]
+        x = logits.reshape(-1, V).contiguous()
+        t = target.reshape(-1).contiguous()
+        n = _all_reduce_sum(ops.gh_count_valid(t, V, ignore_index), group)
+        loss, grad = ops.gh_ce_fwd_bwd_shard(x, t, n, ignore_index, reduction, z)
+        loss = _all_reduce_sum(loss, group)
+        ctx.shape = logits.shape
+        ctx.save_for_backward(grad)
+        return loss
+
+    @staticmethod
+    def backward(ctx, g):
+        (grad,) = ctx.saved_tensors
+        return _scaled(grad, g).view(ctx.shape), None, None, None, None, None, None
+
+
+def data_parallel_cross_entropy(logits, target, ignore_index: int = -100, reduction: str = "mean",
+                                z_loss_multiplier: float = 0.0, group=None, ops=None):
+    """``cross_entropy`` of the whole batch whose shard ``logits`` / ``target``
+    this rank holds (the mean divides by the valid count over all ranks)."""
+    return _DPCrossEntropy.apply(logits, target, ignore_index, reduction, float(z_loss_multiplier), group,
+                                 _ops(ops))
+
+
+class _DPLinearCE(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, inputs, weight, target, ignore_index, reduction, z, accum, group, ops):
+        t = target.contiguous()
+        n = _all_reduce_sum(ops.gh_count_valid(t, weight.shape[0], ignore_index), group)
+        loss, dX, dW = ops.gh_linear_ce_shard(inputs.contiguous(), weight.contiguous(), t, n, ignore_index,
+                                              reduction, z, 0, accum)
+        loss = _all_reduce_sum(loss, group)
+        dW = _all_reduce_sum(dW, group)
+        ctx.save_for_backward(dX, dW)
+        return loss
+
+    @staticmethod
+    def backward(ctx, g):
+        dX, dW = ctx.saved_tensors
+        return (_scaled(dX, g) if ctx.needs_input_grad[0] else None,
+                _scaled(dW, g) if ctx.needs_input_grad[1] else None, None, None, None, None, None, None, None)
+
+
+def data_parallel_chunked_linear_cross_entropy(inputs, weight, target, ignore_index: int = -100,
+                                               reduction: str = "mean", z_loss_multiplier: float = 0.0,
+                                               grad_weight_accum_dtype: str = "fp32", group=None, ops=None):
+    """``chunked_linear_cross_entropy`` of the whole batch whose rows ``inputs`` /
+    ``target`` this rank holds, with the weight replicated: the weight gradient
+    is summed over the ranks (in the weight dtype)."""
+    return _DPLinearCE.apply(inputs, weight, target, ignore_index, reduction, float(z_loss_multiplier),
+                             grad_weight_accum_dtype, group, _ops(ops))

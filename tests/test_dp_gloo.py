@@ -1,0 +1,107 @@
+"""The data-parallel cross-entropy's collective steps on two gloo ranks (CPU).
+
+Each rank holds half of a batch.  The library's shard entry points are
+replaced by float64 PyTorch stand-ins with the same contract (count the valid
+targets; divide by the total count passed in), so what runs here is exactly
+the wrapper's sequence of all-reduces: the valid counts summed before the
+shard call, the losses and the weight gradients summed after it.  Every rank
+must then hold the full batch's mean loss, its own rows of the full batch's
+input/logits gradient, and the full weight gradient.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class _HostOps:
+    """float64 stand-ins for gh_count_valid / gh_ce_fwd_bwd_shard / gh_linear_ce_shard."""
+
+    @staticmethod
+    def gh_count_valid(t, V, ii):
+        return torch.tensor((t != ii).sum().item(), dtype=torch.int64)
+
+    @staticmethod
+    def _rows(x, t, ii, z):
+        valid = t != ii
+        tt = torch.where(valid, t, torch.zeros_like(t))
+        lse = torch.logsumexp(x, dim=1)
+        rl = torch.where(valid, lse - x.gather(1, tt[:, None])[:, 0] + z * lse * lse, torch.zeros_like(lse))
+        g = torch.softmax(x, dim=1) * (1 + 2 * z * lse)[:, None]
+        g[torch.arange(x.shape[0]), tt] -= 1.0
+        return rl, g * valid[:, None]
+
+    @classmethod
+    def gh_ce_fwd_bwd_shard(cls, x, t, n, ii, reduction, z):
+        rl, g = cls._rows(x, t, ii, z)
+        scale = 1.0 / max(int(n), 1) if reduction == "mean" else 1.0
+        return (rl.sum() * scale).reshape(()), g * scale
+
+    @classmethod
+    def gh_linear_ce_shard(cls, X, W, t, n, ii, reduction, z, chunk, accum):
+        loss, G = cls.gh_ce_fwd_bwd_shard(X @ W.T, t, n, ii, reduction, z)
+        return loss, G @ W, G.T @ X
+
+
+def _batch(seed=0, N=24, D=6, V=17):
+    g = torch.Generator().manual_seed(seed)
+    X = torch.randn(N, D, generator=g, dtype=torch.float64)
+    W = torch.randn(V, D, generator=g, dtype=torch.float64) * 0.3
+    t = torch.randint(0, V, (N,), generator=g)
+    t[::5] = -100
+    t[1] = -100  # more ignored rows on rank 0 than on rank 1
+    return X, W, t
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+    from lm_head_cross_gh_b200 import functional as GF
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    X, W, t = _batch()
+    rows = slice(rank * 12, (rank + 1) * 12)
+    # standalone CE on the logits shard
+    logits = (X @ W.T)[rows].clone().requires_grad_(True)
+    loss = GF.data_parallel_cross_entropy(logits, t[rows], -100, "mean", 1e-3, ops=_HostOps)
+    loss.backward()
+    # linear CE with a replicated weight
+    Xs = X[rows].clone().requires_grad_(True)
+    Wr = W.clone().requires_grad_(True)
+    lin = GF.data_parallel_chunked_linear_cross_entropy(Xs, Wr, t[rows], -100, "mean", 1e-3, ops=_HostOps)
+    lin.backward()
+    out.put((rank, loss.item(), logits.grad, lin.item(), Xs.grad, Wr.grad))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_data_parallel_cross_entropy():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=180) for _ in procs), key=lambda r: r[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # the full batch on one process, same stand-in arithmetic
+    X, W, t = _batch()
+    Xf, Wf = X.clone().requires_grad_(True), W.clone().requires_grad_(True)
+    n = int((t != -100).sum())
+    lf, Gf = _HostOps.gh_ce_fwd_bwd_shard(X @ W.T, t, n, -100, "mean", 1e-3)
+    for rank, loss, glog, lin, gx, gw in res:
+        rows = slice(rank * 12, (rank + 1) * 12)
+        assert loss == pytest.approx(lf.item(), rel=1e-12)
+        assert torch.allclose(glog, Gf[rows], rtol=1e-12, atol=1e-15)
+        assert lin == pytest.approx(lf.item(), rel=1e-12)
+        assert torch.allclose(gx, (Gf @ W)[rows], rtol=1e-10, atol=1e-13)
+        assert torch.allclose(gw, Gf.T @ X, rtol=1e-10, atol=1e-13)

@@ -1,0 +1,93 @@
+"""Data-parallel shard entry points on one GPU.
+
+gh_ce_fwd_bwd_shard / gh_linear_ce_shard divide the mean by a total count the
+caller passes; with a total of twice the local count the loss and gradients
+are the oracle's for scale 1 / (2 n_valid).  With the local count they are
+bitwise those of gh_ce_fwd_bwd / gh_linear_ce.  The data-parallel functional
+wrappers on a one-rank NCCL group (the all-reduces are then identities) give
+the same results as the single-process functions.
+"""
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import gh_synth
+import lm_head_cross_gh_b200 as gh
+import oracle
+from ce_check import check_grad, check_loss, grad_to_f64, loss_atol, row_eps, to_device
+from lm_head_cross_gh_b200 import functional as GF
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("path", ["rows", "ring"])
+def test_ce_shard_divides_by_the_given_total(cuda_device, monkeypatch, path):
+    monkeypatch.setenv("GH_CE_PATH", path)
+    p = gh_synth.ce_normal(300, 5003, 3.0, dtype="bf16", ignore_frac=0.1, z_loss=1e-4, seed=11)
+    x, t = to_device(p)
+    n_local = int((p.targets != p.ignore_index).sum())
+    assert gh.gh_count_valid(t, p.V, p.ignore_index).item() == n_local
+    total = torch.tensor(2 * n_local, dtype=torch.int64, device="cuda")
+    loss, grad = gh.gh_ce_fwd_bwd_shard(x, t, total, p.ignore_index, "mean", 1e-4)
+    torch.cuda.synchronize()
+    xv = p.values_f32().astype(np.float64)
+    scale = 1.0 / (2 * n_local)
+    lse, rl, g_ref = oracle.ce_rows(xv, p.targets, p.ignore_index, 1e-4, scale)
+    valid = p.targets != p.ignore_index
+    eps = row_eps(xv)
+    check_loss(loss.item(), float(rl.sum()) * scale, loss_atol(eps, lse, valid, "sum") * scale, "shard loss")
+    check_grad(grad_to_f64(grad), g_ref, "bf16", scale, p.targets, p.ignore_index, eps, "shard grad")
+    own = torch.tensor(n_local, dtype=torch.int64, device="cuda")
+    l1, g1 = gh.gh_ce_fwd_bwd_shard(x, t, own, p.ignore_index, "mean", 1e-4)
+    l2, g2 = gh.gh_ce_fwd_bwd(x, t, p.ignore_index, "mean", 1e-4)
+    torch.cuda.synchronize()
+    assert l1.item() == l2.item() and torch.equal(g1.view(torch.int16), g2.view(torch.int16))
+
+
+def test_linear_ce_shard_with_the_local_count_is_linear_ce(cuda_device):
+    q = gh_synth.linear_ce_normal(700, 128, 3001, chunk=256, ignore_frac=0.05, w_sigma=0.05, z_loss=1e-4, seed=12)
+    X = torch.from_numpy(q.inputs.view(np.int16)).cuda().view(torch.bfloat16)
+    W = torch.from_numpy(q.weight.view(np.int16)).cuda().view(torch.bfloat16)
+    t = torch.from_numpy(q.targets).cuda()
+    n = gh.gh_count_valid(t, q.V, -100)
+    a = gh.gh_linear_ce_shard(X, W, t, n, -100, "mean", 1e-4, 256, "fp32")
+    b = gh.gh_linear_ce(X, W, t, -100, "mean", 1e-4, 256, "fp32")
+    torch.cuda.synchronize()
+    assert a[0].item() == b[0].item() and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_data_parallel_wrappers_on_one_rank(cuda_device):
+    import torch.distributed as dist
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
+    try:
+        p = gh_synth.ce_normal(400, 2003, 3.0, dtype="bf16", ignore_frac=0.1, z_loss=1e-4, seed=13)
+        x, t = to_device(p)
+        xa, xb = x.clone().requires_grad_(True), x.clone().requires_grad_(True)
+        la = GF.data_parallel_cross_entropy(xa, t, -100, "mean", 1e-4)
+        lb = GF.cross_entropy(xb, t, -100, "mean", 1e-4)
+        (la + lb).backward()
+        torch.cuda.synchronize()
+        assert la.item() == lb.item() and torch.equal(xa.grad, xb.grad)
+
+        q = gh_synth.linear_ce_normal(512, 128, 3001, chunk=0, ignore_frac=0.05, w_sigma=0.05, seed=14)
+        X = torch.from_numpy(q.inputs.view(np.int16)).cuda().view(torch.bfloat16)
+        W = torch.from_numpy(q.weight.view(np.int16)).cuda().view(torch.bfloat16)
+        tq = torch.from_numpy(q.targets).cuda()
+        Xa, Wa = X.clone().requires_grad_(True), W.clone().requires_grad_(True)
+        Xb, Wb = X.clone().requires_grad_(True), W.clone().requires_grad_(True)
+        ma = GF.data_parallel_chunked_linear_cross_entropy(Xa, Wa, tq)
+        mb = GF.chunked_linear_cross_entropy(Xb, Wb, tq)
+        (ma + mb).backward()
+        torch.cuda.synchronize()
+        assert ma.item() == mb.item()
+        assert torch.equal(Xa.grad, Xb.grad) and torch.equal(Wa.grad, Wb.grad)
+    finally:
+        dist.destroy_process_group()
