@@ -5,7 +5,7 @@
  *
  *  - gh_ce_fwd_bwd: `cross_entropy` — materialised [B, V] logits and [B]
  *    targets; the summed (or mean) loss with optional z-loss and the logits
- *    gradient, both from one pass that streams each row.  nuvec
+ *    gradient, both from the same call (one read of each row from HBM).  nuvec
  *    FastOp::CrossEntropy gives the row loss logsumexp(x) - x[target]
  *    (float32) and FastOp::CrossEntropyVjp its logits gradient.
  *  - gh_ce_fwd: the same loss without the gradient (evaluation; Gpt2 `loss`,
