@@ -792,16 +792,7 @@ gh_status_t ce_ring_launch(const CeArgs& a, int es, int grid, cudaStream_t strea
   } else {
     kern = ring_kernel_for(es, a.mode);
   }
-  static bool raised[64][2][4] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GH_ERR_CUDA;
-  const int kv = es == 4, km = a.mode == kModeFwdBwd && long_rows ? 3 : a.mode;
-  if (dev < 64 && !raised[dev][kv][km]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, ce_ring_smem_bytes()) !=
-        cudaSuccess)
-      return GH_ERR_CUDA;
-    raised[dev][kv][km] = true;
-  }
+  if (ensure_smem_limit(kern, ce_ring_smem_bytes()) != cudaSuccess) return GH_ERR_CUDA;
   ProfileScope prof(a.profile_kind, stream);
   note_launch();
   return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kRingThreads), ce_ring_smem_bytes(), stream, 1,

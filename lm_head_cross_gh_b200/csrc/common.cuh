@@ -3,6 +3,10 @@
 // with no CUDA C++ spelling.
 #pragma once
 
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include <cstdint>
 #include <utility>
 #include <cuda_runtime.h>
@@ -239,6 +243,25 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 
 // Launch `kern` on `stream` with programmatic stream serialisation (and a
 // cluster dimension when cluster > 1).
+// Raise a kernel's dynamic shared memory limit to `bytes`, once per (kernel,
+// device): the attribute belongs to the device's context, and host threads may
+// launch concurrently.
+template <typename... KArgs>
+inline cudaError_t ensure_smem_limit(void (*kern)(KArgs...), int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;  // (kernel, device)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const void* key = reinterpret_cast<const void*>(kern);
+  std::lock_guard<std::mutex> g(mu);
+  for (const auto& d : done)
+    if (d.first == key && d.second == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.emplace_back(key, dev);
+  return e;
+}
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                               int cluster, Args&&... args) {

@@ -110,12 +110,7 @@ template <bool A_MN, bool B_MN>
 gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
                         const sm100::GemmArgs& g, int kind, cudaStream_t stream) {
   auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm100::kGemmSmem);
-  });
-  if (attr_err != cudaSuccess) return GH_ERR_CUDA;
+  if (ensure_smem_limit(kern, sm100::kGemmSmem) != cudaSuccess) return GH_ERR_CUDA;
   const int tiles = g.tiles_m * g.tiles_n * g.k_splits;
   if (tiles == 0) return GH_OK;
   const int grid = std::min(tiles, sm_count());
