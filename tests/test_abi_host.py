@@ -83,3 +83,30 @@ def test_python_binding_validates_before_calling():
     t = torch.zeros(4, dtype=torch.int64)
     with pytest.raises(ValueError):
         gh.gh_ce_fwd_bwd(x, t)  # CPU tensors are refused; no CPU fallback exists
+
+
+def test_newer_entry_points_reject_bad_arguments_on_host(L):
+    bad = gh.GH_ERR_INVALID_ARG
+    lg, tg, out = FAKE, FAKE + (1 << 32), FAKE + (2 << 32)
+    # gh_ce_fwd
+    assert L.gh_ce_fwd(lg, tg, -1, 100, gh.GH_BF16, -100, 0, 0.0, out, None, None) == bad
+    assert L.gh_ce_fwd(lg, tg, 16, 100, gh.GH_BF16, -100, 0, 0.0, None, None, None) == bad
+    assert L.gh_ce_fwd(lg, tg, 16, 100, gh.GH_BF16, -100, 0, 0.0, out, out + 2, None) == bad  # row_loss misaligned
+    # gh_selective_log_softmax
+    assert L.gh_selective_log_softmax(lg, tg, 16, 0, gh.GH_BF16, out, None) == bad
+    assert L.gh_selective_log_softmax(lg, None, 16, 100, gh.GH_BF16, out, None) == bad
+    assert L.gh_selective_log_softmax(lg, tg, 16, 100, 9, out, None) == bad
+    # gh_ce_vjp
+    assert L.gh_ce_vjp(lg, tg, 16, 100, gh.GH_BF16, -100, None, out, FAKE + (3 << 32), None) == bad
+    assert L.gh_ce_vjp(lg, tg, 16, 100, gh.GH_BF16, -100, out, out, lg + 64, None) == bad  # partial overlap
+    # gh_count_valid
+    assert L.gh_count_valid(tg, -1, 100, -100, out, None) == bad
+    assert L.gh_count_valid(tg, 16, 100, -100, out + 4, None) == bad
+    # shard entry points need an aligned total count
+    assert L.gh_ce_fwd_bwd_shard(lg, tg, 16, 100, gh.GH_BF16, -100, 0, 0.0, None, out, FAKE + (3 << 32),
+                                 None) == bad
+    assert L.gh_linear_ce_shard(lg, FAKE + (4 << 32), tg, 64, 64, 100, 0, 0, -100, 0, 0.0, out + 4, out,
+                                FAKE + (5 << 32), FAKE + (6 << 32), None) == bad
+    # gh_chunked_linear_loss needs a callback
+    assert L.gh_chunked_linear_loss(lg, FAKE + (4 << 32), 64, 64, 100, 0, 0, gh.CHUNK_LOSS_FN(), None, out,
+                                    FAKE + (5 << 32), FAKE + (6 << 32), None) == bad
