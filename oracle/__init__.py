@@ -34,7 +34,7 @@ forms, invariants, finite differences, a materialised brute force and
 ``torch.nn.functional.cross_entropy`` (the PyTorch routine the z-free,
 unchunked case reduces to).
 """
-from .ce import (bf16_round, cross_entropy, ce_rows, n_valid_and_scale,
+from .ce import (bf16_round, cross_entropy, ce_rows, ce_vjp, n_valid_and_scale,
                  selective_log_softmax)
 from .linear_ce import linear_cross_entropy, linear_cross_entropy_materialised
 
@@ -42,6 +42,7 @@ __all__ = [
     "bf16_round",
     "cross_entropy",
     "ce_rows",
+    "ce_vjp",
     "n_valid_and_scale",
     "selective_log_softmax",
     "linear_cross_entropy",

@@ -132,3 +132,27 @@ def selective_log_softmax(logits: np.ndarray, index: np.ndarray) -> np.ndarray:
     m = x2.max(axis=1)
     lse = m + np.log(np.exp(x2 - m[:, None]).sum(axis=1))
     return (x2[np.arange(x2.shape[0]), i2] - lse).reshape(lead)
+
+
+def ce_vjp(logits: np.ndarray, targets: np.ndarray, ignore_index: int, g: np.ndarray) -> np.ndarray:
+    """Vector-Jacobian product of the per-row loss ``lse - x[target]``.
+
+    nuvec ``FastOp::CrossEntropyVjp``: for an upstream gradient ``g[r]`` of row
+    r's loss, the logits gradient is ``g[r] * (softmax(x[r]) - onehot(t[r]))``;
+    rows whose target equals ``ignore_index`` have no loss and a zero gradient.
+    """
+    x = np.asarray(logits, dtype=np.float64)
+    t = np.asarray(targets, dtype=np.int64)
+    gv = np.asarray(g, dtype=np.float64)
+    rows, V = x.shape
+    valid = t != ignore_index
+    if ((t[valid] < 0) | (t[valid] >= V)).any():
+        raise ValueError("target outside [0, V)")
+    m = x.max(axis=1)
+    p = np.exp(x - m[:, None])
+    p /= p.sum(axis=1, keepdims=True)
+    vr = np.nonzero(valid)[0]
+    p[vr, t[vr]] -= 1.0
+    out = p * gv[:, None]
+    out[~valid] = 0.0
+    return out

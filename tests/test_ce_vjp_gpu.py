@@ -1,8 +1,8 @@
 """GPU parity of gh_ce_vjp (the per-row cross-entropy's logits gradient for an
 upstream gradient per row, from the forward's row loss) against the oracle.
 
-Reference: for a valid row, grad = g_r * (softmax(x_r) - onehot(t_r)), the
-oracle's z-free, unscaled row gradient times g_r; ignored rows are zero.
+Reference: ``oracle.ce_vjp`` -- for a valid row, grad = g_r * (softmax(x_r) -
+onehot(t_r)); ignored rows are zero.
 
 Tolerance per element: one rounding of the output (2^-8 |ref| for bf16, 2e-5
 |ref| for fp32) plus |g_r| p_rj times the relative error of exp(x - lse):
@@ -26,8 +26,8 @@ pytestmark = pytest.mark.gpu
 
 def reference(p, g):
     x = p.values_f32().astype(np.float64)
-    lse, _, G = oracle.ce_rows(x, p.targets, p.ignore_index, 0.0, 1.0)
-    return G * g[:, None], lse, x
+    lse, _, _ = oracle.ce_rows(x, p.targets, p.ignore_index, 0.0, 1.0, with_grad=False)
+    return oracle.ce_vjp(x, p.targets, p.ignore_index, g), lse, x
 
 
 def check(p, g, out, what, row_loss=None):

@@ -244,3 +244,40 @@ def test_selective_log_softmax_equals_negative_row_loss():
     x, t = _rand_problem(12, 50, seed=12, ignore_frac=0.0)
     r = oracle.cross_entropy(x, t, reduction="sum")
     np.testing.assert_allclose(oracle.selective_log_softmax(x, t), -r["row_loss"], rtol=1e-14)
+
+
+# -- the VJP ------------------------------------------------------------------
+
+def test_vjp_matches_central_differences_of_the_weighted_row_losses():
+    # d/dx sum_r g_r * (lse_r - x_{r,t_r}) by central differences, ignored rows included
+    x, t = _rand_problem(5, 7, seed=21, ignore_frac=0.4)
+    g = np.random.default_rng(3).normal(size=5)
+    out = oracle.ce_vjp(x, t, -100, g)
+
+    def f(xx):
+        _, rl, _ = oracle.ce_rows(xx, t, -100, 0.0, 1.0, with_grad=False)
+        return float((g * rl).sum())
+
+    h = 1e-6
+    fd = np.zeros_like(x)
+    for i in range(x.shape[0]):
+        for j in range(x.shape[1]):
+            xp = x.copy(); xp[i, j] += h
+            xm = x.copy(); xm[i, j] -= h
+            fd[i, j] = (f(xp) - f(xm)) / (2 * h)
+    np.testing.assert_allclose(out, fd, rtol=1e-7, atol=1e-8)
+    assert not out[t == -100].any()
+
+
+def test_vjp_matches_torch_autograd_and_the_scaled_row_gradient():
+    x, t = _rand_problem(9, 13, seed=22, ignore_frac=0.2)
+    g = np.random.default_rng(4).uniform(-2, 2, size=9)
+    xt = torch.tensor(x, requires_grad=True)
+    tt = torch.tensor(np.where(t == -100, -100, t))
+    rl = torch.nn.functional.cross_entropy(xt, tt, ignore_index=-100, reduction="none")
+    (rl * torch.tensor(g)).sum().backward()
+    out = oracle.ce_vjp(x, t, -100, g)
+    np.testing.assert_allclose(out, xt.grad.numpy(), rtol=1e-12, atol=1e-14)
+    # with z = 0 the unscaled row gradient times g is the VJP
+    _, _, G = oracle.ce_rows(x, t, -100, 0.0, 1.0)
+    np.testing.assert_allclose(out, G * g[:, None], rtol=1e-12, atol=1e-15)
