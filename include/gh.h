@@ -159,7 +159,7 @@ gh_status_t gh_linear_ce_shard(const void* inputs, const void* weight, const int
 
 /*
  * gh_ce_fwd — the cross-entropy loss of gh_ce_fwd_bwd without its gradient:
- * the evaluation form (a forward with no tape and no gradients), reading the
+ * the evaluation form (forward only, nothing kept for a backward), reading the
  * logits once.
  *
  *   logits, targets, B, V, dtype, ignore_index, reduction, z_mult, loss
@@ -178,8 +178,8 @@ gh_status_t gh_ce_fwd(const void* logits, const int64_t* targets, int64_t B, int
  * gradient per row (nuvec FastOp::CrossEntropyVjp: logits, targets, the
  * forward's row loss and g):
  *     grad_j = g_r (exp(x_j - lse_r) - [j == t_r]),   lse_r = row_loss_r + x_{r,t_r}
- * The forward's row loss carries lse, so the gradient is one streaming pass
- * with no reduction.
+ * The forward's row loss carries lse, so the gradient takes one sweep over
+ * each row with no reduction.
  *
  *   logits, targets, B, V, dtype, ignore_index  as for gh_ce_fwd_bwd.
  *   row_loss  [B] float32, device: lse - x_t per row without z-loss, as

@@ -1,7 +1,8 @@
-// Standalone streaming cross-entropy, forward and backward in one call
-// (Greyhound functional API, `cross_entropy`: "summed loss and logits
-// gradient in one streaming pass"; nuvec FastOp::CrossEntropy /
-// CrossEntropyVjp for the row loss and its gradient).
+// Standalone cross-entropy, forward and backward in one call (Greyhound
+// functional API, `cross_entropy`: the summed or mean loss and the logits
+// gradient from one call; nuvec FastOp::CrossEntropy / CrossEntropyVjp for the
+// row loss and its gradient).  The ring pipelines in ce_ring.cu take batches
+// of 8 rows per SM or more; the row kernel below takes the smaller ones.
 //
 // Kernels, in launch order on the caller's stream:
 //   ce_count_kernel  n_valid = #{t != ignore_index}; flags targets outside [0, V)

@@ -5,7 +5,7 @@
 // The forward's row loss is lse - x_t, so lse = loss + x_t comes back from one
 // element of the row and no reduction is needed: the gradient
 //     grad_j = g (exp(x_j - lse) - [j == t])
-// is a single streaming pass, one read and one write of every logit.  Rows
+// takes one read and one write of every logit, in a single sweep per row.  Rows
 // whose target equals ignore_index (or lies outside [0, V)) get a zero row.
 //
 // ce_vjp_kernel: persistent CTAs of 512 threads, rows round-robin.  Thread 0

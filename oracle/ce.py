@@ -1,8 +1,8 @@
 """Float64 oracle for the standalone cross-entropy (test infrastructure only).
 
 Follows the Greyhound functional API page, ``cross_entropy`` (parameters
-``ignore_index``, ``reduction``, ``z_loss_multiplier``; "one streaming pass"
-yielding the summed loss and the logits gradient) and nuvec
+``ignore_index``, ``reduction``, ``z_loss_multiplier``; the loss and the logits
+gradient come out of the same call) and nuvec
 ``FastOp::CrossEntropy`` / ``FastOp::CrossEntropyVjp`` (row loss
 ``logsumexp(logits) - logits[target]`` and its gradient).
 
@@ -12,10 +12,10 @@ Notation: for a row x with target t and ``lse = log sum_j exp(x_j)``,
     grad_j   = scale * ((1 + 2 z lse) * exp(x_j - lse) - [j == t])
     scale    = 1 / max(n_valid, 1)  for "mean",  1 for "sum"
 
-and ignored rows contribute neither loss nor gradient.  The z-loss form
-``z * lse**2`` is the reading of "penalizes large log-partition function
-values" that the problem statement fixes; its derivative ``2 z lse * p_j``
-gives the ``(1 + 2 z lse)`` factor.
+and ignored rows contribute neither loss nor gradient.  The page describes the
+z-loss only as a penalty on large log-partition values; the form
+``z * lse**2`` is the one the problem statement fixes, and its derivative
+``2 z lse * p_j`` gives the ``(1 + 2 z lse)`` factor.
 """
 from __future__ import annotations
 
