@@ -253,10 +253,12 @@ def gh_linear_ce_shard(inputs, weight, targets, n_valid_total, ignore_index: int
     import torch
     _need(inputs.dim() == 2 and weight.dim() == 2 and inputs.shape[1] == weight.shape[1], "shapes")
     _need(inputs.dtype == torch.bfloat16 and weight.dtype == torch.bfloat16, "inputs/weight must be bfloat16")
+    _need(inputs.is_cuda and weight.is_cuda and inputs.is_contiguous() and weight.is_contiguous(), "layout")
     _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
           and targets.shape == (inputs.shape[0],), "targets: contiguous CUDA int64 [N]")
     _need(n_valid_total.dtype == torch.int64 and n_valid_total.numel() == 1 and n_valid_total.is_cuda,
           "n_valid_total: CUDA int64 scalar")
+    _need(reduction in GH_REDUCTION and accum in GH_ACCUM, "reduction / accum")
     N, D = inputs.shape
     V = weight.shape[0]
     if grad_inputs is None:
