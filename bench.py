@@ -2,23 +2,33 @@
 """Throughput of the next-token cross-entropy hot path on B200.
 
 One JSON line (rank 0).  Default workload: standalone CE forward+backward on
-GPT-2-shaped bf16 logits [8192, 50257] (2% ignored, mean, z-loss 1e-4); the
-same line carries the chunked linear-CE on the GPT-2 small tied head
-([8192, 768] x [50257, 768], chunk 2048, fp32 accumulation) under "linear_ce".
+GPT-2-shaped bf16 logits [8192, 50257] (2% ignored, mean, z-loss 1e-4).  The
+same line carries, each under its own key with its own roofline and clocks:
+
+* "linear_ce": chunked linear-CE on the GPT-2 small tied head
+  ([8192, 768] x [50257, 768], chunk 2048, fp32 accumulation);
+* "linear_ce_llama3_8b": the Llama-3-8B head ([16384, 4096] x [128256, 4096],
+  5% ignored, chunk 4096, fp32 accumulation, z-loss 1e-4);
+* "ce_large_vocab": CE forward+backward on bf16 [4096, 262144] Student-t logits
+  with spikes (sum, z-loss 1e-4).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
+                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline] [--no-extra]
 
 Timing: CUDA events on the launching stream around exactly K steps, bracketed
 by a barrier and a device synchronise, max over ranks.  Inputs are larger than
 L2 (126 MB) for the timed workloads, so no flush runs between steps.  Kernel
-durations for the roofline come from libgh's own event pairs around the
-dominant kernel, recorded over a separate run of the same K steps just before
-the timed region (event records between kernels would hide the programmatic
-launch overlap, so they stay out of the region that gives `value`).  With N > 1 each rank
+durations for the roofline come from libgh's own event pairs around each
+kernel, recorded over a separate run of the same K steps just before the timed
+region (event records between kernels would hide the programmatic launch
+overlap, so they stay out of the region that gives `value`).  The CE roofline
+is the dominant kernel's algorithmic bytes over its launch time against the
+measured copy bandwidth; the linear-CE roofline is the whole step's 6 N V D
+FLOPs over the step time against the dense bf16 matmul peak (burst for short
+timed regions), with each GEMM's own rate alongside.  With N > 1 each rank
 processes its own batch (seed = rank); nothing is exchanged (weak scaling).
 ``--impl reference`` times the float64 CPU oracle on a bounded sample of the
-same workload (rank 0 only).
+same workload (rank 0 only), on all host cores.
 """
 from __future__ import annotations
 
@@ -26,7 +36,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import statistics
 import sys
 import threading
@@ -85,19 +94,20 @@ def source_digest(files):
     return h.hexdigest()[:12]
 
 
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+
+
 def profiled_traffic(kernel, digest, workload):
-    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu summary
-    (`profiles/<kernel>_*.md`; for the forward ring `<kernel>` names the
-    operation too), if one was taken of the current source."""
-    import glob
-    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*.md"))):
-        txt = open(p).read()
-        m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", txt)
-        if not m_sha or m_sha.group(1) != digest:
-            continue
-        for m in re.finditer(r"workload:\s*(\S+)\s*\ntraffic_bytes_per_launch:\s*([0-9.eE+]+)", txt):
-            if m.group(1) == workload:
-                return float(m.group(2))
+    """DRAM bytes per launch of `kernel` on `workload` (dram__bytes_read.sum +
+    dram__bytes_write.sum of one ncu capture), from ``profiles/traffic.json``,
+    if that capture was taken of the current source (same digest)."""
+    if not os.path.exists(TRAFFIC_JSON):
+        return None
+    with open(TRAFFIC_JSON) as f:
+        entries = json.load(f).get("entries", [])
+    for e in entries:
+        if e["kernel"] == kernel and e["source_sha"] == digest and e["workload"] == workload:
+            return float(e["traffic_bytes_per_launch"])
     return None
 
 
@@ -289,16 +299,39 @@ def ce_config(p, op):
             "l2": f"inputs larger than L2 ({p.B * p.V * (4 if p.dtype == 'f32' else 2) / 1e6:.0f} MB); no flush"}
 
 
-def ce_oracle_rows(p, op, rows):
-    """The float64 oracle on a sample of rows, for the operation `op`."""
+ORACLE_BLOCK_ROWS = 16  # rows per task of the threaded CE oracle
+
+
+def host_threads() -> int:
+    """Host cores this process may use."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def ce_oracle_rows(p, op, rows, threads=1):
+    """The float64 oracle on a sample of rows, for the operation `op`; blocks of
+    rows run on `threads` host threads (numpy releases the GIL in its loops)."""
     import numpy as np
     import oracle
-    x = p.values_f32(rows).astype(np.float64)
-    if op == "select":
-        oracle.selective_log_softmax(x, select_index(p.targets[rows]))
+    _, scale = oracle.n_valid_and_scale(p.targets, p.ignore_index, p.reduction, p.V)
+
+    def block(r):
+        x = p.values_f32(r).astype(np.float64)
+        if op == "select":
+            oracle.selective_log_softmax(x, select_index(p.targets[r]))
+        else:
+            oracle.ce_rows(x, p.targets[r], p.ignore_index, p.z_loss, scale, with_grad=op == "fwd_bwd")
+
+    blocks = [rows[i:i + ORACLE_BLOCK_ROWS] for i in range(0, len(rows), ORACLE_BLOCK_ROWS)]
+    if threads <= 1 or len(blocks) <= 1:
+        for b in blocks:
+            block(b)
     else:
-        _, scale = oracle.n_valid_and_scale(p.targets, p.ignore_index, p.reduction, p.V)
-        oracle.ce_rows(x, p.targets[rows], p.ignore_index, p.z_loss, scale, with_grad=op == "fwd_bwd")
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(block, blocks))
     return len(rows)
 
 
@@ -366,8 +399,8 @@ class CeCase:
         import numpy as np
         return np.arange(min(self.p.B, budget_rows))
 
-    def run_oracle(self, rows):
-        return ce_oracle_rows(self.p, self.op, rows)
+    def run_oracle(self, rows, threads=1):
+        return ce_oracle_rows(self.p, self.op, rows, threads)
 
 
 def linear_config(p):
@@ -423,8 +456,9 @@ class LinearCase:
         import numpy as np
         return np.arange(min(self.p.N, budget_rows))
 
-    def run_oracle(self, rows):
-        """Oracle on a row sample: the chunk's logits, CE and both gradient GEMMs (float64)."""
+    def run_oracle(self, rows, threads=1):
+        """Oracle on a row sample: the chunk's logits, CE and both gradient GEMMs
+        (float64; numpy's BLAS threads, whatever `threads` says)."""
         import numpy as np
         import gh_synth
         import oracle
@@ -437,8 +471,10 @@ class LinearCase:
         return len(rows)
 
 
-KERNEL_OF = {"ce": "ce_row", "linear": "logits_gemm"}
 CE_RING_MIN_ROWS_PER_SM = 8  # the library's switch from the row kernel to the ring pipelines
+GEMM_KINDS = ("logits_gemm", "dx_gemm", "dw_gemm")
+LINEAR_KINDS = GEMM_KINDS + ("chunk_ce",)
+SUSTAINED_AFTER_S = 2.0  # a timed region at least this long is compared with the sustained matmul peak
 
 
 def ce_kernel_of(case, device_index):
@@ -456,6 +492,10 @@ def ce_kernel_of(case, device_index):
     return "ce_row_kernel", ["lm_head_cross_gh_b200/csrc/ce.cu"] + common
 
 
+LINEAR_SOURCES = ["lm_head_cross_gh_b200/csrc/gemm_sm100.cuh", "lm_head_cross_gh_b200/csrc/linear_ce.cu",
+                  "lm_head_cross_gh_b200/csrc/common.cuh"]
+
+
 def time_steps(case, dist, steps, warmup, clocks=None):
     """Kernel durations for the roofline, then exactly `steps` timed steps.
 
@@ -471,7 +511,7 @@ def time_steps(case, dist, steps, warmup, clocks=None):
         case.step()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    kinds = ["ce_row"] if case.kind == "ce" else ["logits_gemm", "chunk_ce", "dx_gemm", "dw_gemm"]
+    kinds = ["ce_row"] if case.kind == "ce" else list(LINEAR_KINDS)
     for rep in range(2):
         gh.gh_profile_enable(True)
         for _ in range(steps):
@@ -539,27 +579,101 @@ def cpu_threads():
         return 1
 
 
+def oracle_threads(case):
+    """Threads the oracle runs on: one per host core for the CE row loops, the
+    BLAS pool for linear-CE."""
+    return host_threads() if case.kind == "ce" else cpu_threads()
+
+
 def run_oracle_timing(case, budget_rows, reps=1):
+    threads = oracle_threads(case)
     rows = case.cpu_sample(budget_rows)
     t0 = time.perf_counter()
     n = 0
     for _ in range(reps):
-        n += case.run_oracle(rows)
+        n += case.run_oracle(rows, threads)
     dt = time.perf_counter() - t0
-    return n / dt, len(rows), dt
+    return n / dt, len(rows), dt, threads
 
 
-ORACLE_ROWS = {"ce_gpt2": 1024, "ce_large_vocab": 256, "ce_small": 64, "linear_ce_gpt2": 512,
+# Oracle rows per host thread in one timing sample (linear-CE: per sample, BLAS-threaded).
+ORACLE_ROWS = {"ce_gpt2": 1024, "ce_large_vocab": 64, "ce_small": 64, "linear_ce_gpt2": 512,
                "linear_ce_llama3_8b": 32}
 
 
-def linear_summary(case, ms, kern, steps, pk, peak_kind):
-    tot_ms = ms / steps
-    tflops = case.flops_per_step / (tot_ms * 1e-3) / 1e12
-    gemm_ms = sum(kern[k][0] for k in ("logits_gemm", "dx_gemm", "dw_gemm")) / steps
-    gemm_tflops = case.flops_per_step / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
-    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-    return tot_ms, tflops, gemm_ms, gemm_tflops, peak
+def ce_roofline(case, kern, steps, pk, pk_kind, device_index):
+    """The CE kernel's algorithmic bytes over its event-timed launch duration."""
+    k_ms, k_n = kern["ce_row"]
+    k_avg = k_ms / max(k_n, 1)
+    achieved = case.bytes_per_step / (k_avg * 1e-3) / 1e9
+    kname, ksrc = ce_kernel_of(case, device_index)
+    digest = source_digest(ksrc)
+    prefix = kname if kname != "ce_ring_kernel" else f"ce_ring_kernel_{case.op}"
+    return {"bound": "hbm", "kernel": kname, "achieved": achieved,
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+            "traffic": profiled_traffic(prefix, digest, case.p.name), "algorithmic_bytes": case.bytes_per_step,
+            "kernel_ms": k_avg, "peak_source": f"{pk_kind} (copy)", "source_sha": digest}
+
+
+def linear_roofline(case, ms_total, kern, steps, pk, pk_kind):
+    """The whole step's algorithmic FLOPs (6 N V D: logits, dX and dW GEMMs) over
+    the step time, against the dense bf16 matmul peak: the burst figure for a
+    timed region shorter than SUSTAINED_AFTER_S, the sustained one beyond.  Each
+    GEMM's own rate (2 N V D per step over its event-timed launches) and the
+    per-chunk cross-entropy kernels' time are listed alongside."""
+    step_ms = ms_total / steps
+    sustained = ms_total * 1e-3 >= SUSTAINED_AFTER_S and "bf16_tflops_sustained" in pk
+    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    achieved = case.flops_per_step / (step_ms * 1e-3) / 1e12
+    digest = source_digest(LINEAR_SOURCES)
+    parts = {}
+    traffic_step = 0.0
+    for k in LINEAR_KINDS:
+        tot, n = kern.get(k, (0.0, 0))
+        if not n:
+            continue
+        per_ms = tot / n
+        d = {"ms_per_launch": per_ms, "launches_per_step": n / steps, "ms_per_step": tot / steps}
+        if k in GEMM_KINDS:
+            flops = case.flops_per_step / 3.0 * steps / n
+            d["tflops"] = flops / (per_ms * 1e-3) / 1e12
+            d["frac"] = d["tflops"] / peak
+            tr = profiled_traffic(k, digest, case.p.name)
+            d["traffic"] = tr
+            traffic_step = None if (tr is None or traffic_step is None) else traffic_step + tr * n / steps
+        parts[k] = d
+    return {"bound": "tensor", "kernel": "whole step: logits GEMM with its cross-entropy epilogue, "
+                                          "per-chunk finalize, dX and dW GEMMs",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic_step if parts else None, "algorithmic_flops": case.flops_per_step,
+            "step_ms": step_ms, "kernels": parts,
+            "peak_source": f"{pk_kind} bf16 ({'sustained' if sustained else 'burst'})", "source_sha": digest}
+
+
+def measure(case, dist, steps, warmup, pk, pk_kind):
+    """Timed steps of one workload: throughput, roofline, clocks, launches."""
+    clocks = ClockSampler(dist.local)
+    ms, launches, kern = time_steps(case, dist, steps, warmup, clocks)
+    value, ms_max = aggregate(dist, ms, case.tokens * steps)
+    out = {"workload": case.p.name, "value": value, "unit": "tokens/s", "ms_per_step": ms_max / steps,
+           "steps": steps, "gpu_launches": int(launches)}
+    if case.kind == "ce":
+        out["roofline"] = ce_roofline(case, kern, steps, pk, pk_kind, dist.local)
+        out["hbm_gbs_step"] = case.bytes_per_step * steps / (ms * 1e-3) / 1e9
+    else:
+        out["roofline"] = linear_roofline(case, ms_max, kern, steps, pk, pk_kind)
+        out["tflops"] = out["roofline"]["achieved"]
+    out["clocks"] = clocks.summary()
+    return out
+
+
+# Workloads the default CE line also carries (name, steps cap).
+EXTRA_WORKLOADS = (("linear_ce", "linear_ce_gpt2", 20), ("linear_ce_llama3_8b", "linear_ce_llama3_8b", 3),
+                   ("ce_large_vocab", "ce_large_vocab", 20))
+
+
+def make_case(name, seed, dev, op="fwd_bwd"):
+    return CeCase(name, seed, dev, op) if name in CE_WORKLOADS else LinearCase(name, seed, dev)
 
 
 def main():
@@ -573,7 +687,8 @@ def main():
                     help="standalone CE operation timed on a CE workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-linear", action="store_true", help="omit the linear-CE object on the CE line")
+    ap.add_argument("--no-extra", "--no-linear", dest="no_extra", action="store_true",
+                    help="omit the other workloads' objects from the default CE line")
     ap.add_argument("--rows", type=int, default=0, help="use only the first ROWS rows/tokens (profiling cases)")
     ap.add_argument("--launches-only", action="store_true",
                     help="run W + K steps and exit without timing or report (for ncu captures)")
@@ -598,42 +713,27 @@ def main():
     pk, pk_kind = peaks()
 
     is_ce = args.workload in CE_WORKLOADS
-    case = CeCase(args.workload, dist.rank, dev, args.op) if is_ce else LinearCase(args.workload, dist.rank, dev)
+    case = make_case(args.workload, dist.rank, dev, args.op)
     if args.launches_only:
         for _ in range(args.warmup + args.steps):
             case.step()
         torch.cuda.synchronize()
         dist.close()
         return 0
-    clocks = ClockSampler(dist.local)
-    ms, launches, kern = time_steps(case, dist, args.steps, args.warmup, clocks)
-    value, ms_max = aggregate(dist, ms, case.tokens * args.steps)
+    m = measure(case, dist, args.steps, args.warmup, pk, pk_kind)
 
-    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+    out = {"metric": METRIC, "value": m["value"], "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": case.dtype,
            "data": "synthetic (seeded; seed = rank)", "config": case.config()}
     out["config"]["parallelism"] = parallelism(dist.world)
-
+    out["roofline"] = m["roofline"]
     if is_ce:
-        k_ms, k_n = kern["ce_row"]
-        k_avg = k_ms / max(k_n, 1)
-        achieved = case.bytes_per_step / (k_avg * 1e-3) / 1e9
-        kname, ksrc = ce_kernel_of(case, dist.local)
-        digest = source_digest(ksrc)
-        prefix = kname if kname != "ce_ring_kernel" else f"ce_ring_kernel_{case.op}"
-        traffic = profiled_traffic(prefix, digest, case.p.name)
-        out["roofline"] = {"bound": "hbm", "kernel": kname, "achieved": achieved,
-                           "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                           "traffic": traffic, "algorithmic_bytes": case.bytes_per_step,
-                           "kernel_ms": k_avg, "peak_source": f"{pk_kind} (copy)", "source_sha": digest}
-        out["hbm_gbs_step"] = case.bytes_per_step * args.steps / (ms * 1e-3) / 1e9
+        out["hbm_gbs_step"] = m["hbm_gbs_step"]
     else:
-        tot_ms, tflops, gemm_ms, gemm_tflops, peak = linear_summary(case, ms, kern, args.steps, pk, pk_kind)
-        out["tflops"] = tflops
-        out["roofline"] = linear_roofline(case, kern, args.steps, pk, pk_kind)
-    out["gpu_launches"] = int(launches)
-    out["clocks"] = clocks.summary()
+        out["tflops"] = m["tflops"]
+    out["gpu_launches"] = m["gpu_launches"]
+    out["clocks"] = m["clocks"]
 
     if not args.no_e2e:
         k = max(1, min(args.steps, 10))
@@ -642,43 +742,30 @@ def main():
                       "h2d_bytes_per_step": case.h2d, "d2h_bytes_per_step": case.d2h,
                       "path": "pinned host -> device copies, gh C ABI call, loss read back, per step"}
 
-    if is_ce and not args.no_linear and dist.world >= 1:
-        try:
-            lcase = LinearCase("linear_ce_gpt2", dist.rank, dev)
-            lsteps = max(3, min(args.steps, 20))
-            lms, llaunch, lkern = time_steps(lcase, dist, lsteps, args.warmup, None)
-            lms = dist.max(lms)
-            tot_ms, tflops, gemm_ms, gemm_tflops, peak = linear_summary(lcase, lms, lkern, lsteps, pk, pk_kind)
-            out["linear_ce"] = {"workload": lcase.p.name, "value": dist.sum(lcase.tokens * lsteps) / (lms * 1e-3),
-                                "unit": "tokens/s", "ms_per_step": lms / lsteps, "tflops": tflops,
-                                "steps": lsteps, "gpu_launches": int(llaunch),
-                                "roofline": linear_roofline(lcase, lkern, lsteps, pk, pk_kind)}
-            del lcase
-        except Exception as e:  # the CE line stands on its own
-            out["linear_ce"] = {"unavailable": f"{type(e).__name__}: {e}"}
-
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        rows = ORACLE_ROWS[args.workload]
-        v, nrows, dt = run_oracle_timing(case, rows)
-        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1 if is_ce else cpu_threads(),
-                               "kind": "oracle",
-                               "sample": f"first {nrows} rows of the same workload, float64 numpy oracle, "
-                                         f"{dt:.1f} s"}
+        v, nrows, dt, threads = run_oracle_timing(case, ORACLE_ROWS[args.workload] *
+                                                  (host_threads() if is_ce else 1))
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                               "sample": f"first {nrows} rows of the same workload, float64 numpy oracle on "
+                                         f"{threads} host threads, {dt:.1f} s"}
+
+    if is_ce and args.workload == "ce_gpt2" and args.op == "fwd_bwd" and not args.no_extra:
+        del case
+        torch.cuda.empty_cache()
+        for key, name, cap in EXTRA_WORKLOADS:
+            try:
+                extra = make_case(name, dist.rank, dev)
+                st = max(3, min(args.steps, cap))
+                obj = measure(extra, dist, st, args.warmup, pk, pk_kind)
+                obj["config"] = extra.config()
+                out[key] = obj
+                del extra
+            except Exception as e:  # the CE line stands on its own
+                out[key] = {"workload": name, "unavailable": f"{type(e).__name__}: {e}"}
+            torch.cuda.empty_cache()
     if dist.rank == 0:
         print(json.dumps(out), flush=True)
     dist.close()
-
-
-def linear_roofline(case, kern, steps, pk, pk_kind):
-    peak = pk.get("bf16_tflops_sustained") or pk.get("bf16_tflops")
-    gemm_ms = sum(kern[k][0] for k in ("logits_gemm", "dx_gemm", "dw_gemm")) / steps
-    per = {k: kern[k][0] / max(kern[k][1], 1) for k in kern}
-    achieved = case.flops_per_step / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
-    return {"bound": "tensor", "kernel": "tcgen05 GEMMs (logits, dX, dW) per step",
-            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": (achieved / peak) if achieved else None, "traffic": None,
-            "algorithmic_flops": case.flops_per_step, "kernel_ms_per_launch": per,
-            "peak_source": f"{pk_kind} bf16 (sustained)"}
 
 
 def parallelism(world):
@@ -692,35 +779,36 @@ def reference_arm(args, dist):
     is_ce = args.workload in CE_WORKLOADS
 
     class Dummy:
-        pass
+        kind = "ce" if is_ce else "linear"
     case = Dummy()
     if is_ce:
         case.p = make_ce(args.workload, 0)
         case.cpu_sample = lambda n, c=case: __import__("numpy").arange(min(c.p.B, n))
-        case.run_oracle = lambda rows, c=case: ce_oracle_rows(c.p, args.op, rows)
+        case.run_oracle = lambda rows, threads, c=case: ce_oracle_rows(c.p, args.op, rows, threads)
         config = ce_config(case.p, args.op)
     else:
         case.p = make_linear(args.workload, 0)
         case.cpu_sample = lambda n, c=case: __import__("numpy").arange(min(c.p.N, n))
-        case.run_oracle = lambda rows, c=case: LinearCase.run_oracle(c, rows)
+        case.run_oracle = lambda rows, threads, c=case: LinearCase.run_oracle(c, rows, threads)
         config = linear_config(case.p)
     config["parallelism"] = parallelism(1)
-    rows_per_step = max(1, ORACLE_ROWS[args.workload] // 8)
+    threads = oracle_threads(case)
+    rows_per_step = max(1, ORACLE_ROWS[args.workload] // 8) * (threads if is_ce else 1)
     rows = case.cpu_sample(rows_per_step)
     for _ in range(args.warmup):
-        case.run_oracle(rows)
+        case.run_oracle(rows, threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        case.run_oracle(rows)
+        case.run_oracle(rows, threads)
     dt = time.perf_counter() - t0
     value = len(rows) * args.steps / dt
-    cores = 1 if is_ce else cpu_threads()
-    sample = f"first {len(rows)} rows of {case.p.name} per step, float64 numpy oracle"
+    sample = f"first {len(rows)} rows of {case.p.name} per step, float64 numpy oracle on {threads} host threads"
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "f64", "data": "synthetic (seeded)", "config": config,
-           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                            "sample": sample},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0

@@ -40,19 +40,60 @@ _ROW_BLOCK_ELEMS = 1 << 22  # ~4M values per independently seeded block
 # bf16 bit handling (input rounding only)
 # ---------------------------------------------------------------------------
 
+_ROUND_BLOCK = 1 << 20  # values per block of the bf16 rounding
+
+
+def _round_block(u: np.ndarray, out: np.ndarray) -> None:
+    # (u + 0x7FFF + lsb) >> 16 with lsb = bit 16 of u: nearest, ties to even.
+    # Finite float32 patterns are at most 0xFF7FFFFF, so the sum fits 32 bits.
+    t = (u >> 16) & np.uint32(1)
+    t += u
+    t += np.uint32(0x7FFF)
+    t >>= 16
+    out[...] = t
+
+
 def f32_to_bf16(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to bf16 (nearest, ties to even); return uint16 bits."""
+    """Round finite float32 values to bf16 (nearest, ties to even); return uint16 bits.
+
+    Works through the array in blocks (threads over blocks), so no temporary
+    larger than a block is ever allocated."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
-    return r
+    u = x.view(np.uint32).reshape(-1)
+    out = np.empty(u.shape, dtype=np.uint16)
+    starts = range(0, u.size, _ROUND_BLOCK)
+
+    def work(i0: int) -> None:
+        _round_block(u[i0:i0 + _ROUND_BLOCK], out[i0:i0 + _ROUND_BLOCK])
+
+    if u.size <= _ROUND_BLOCK:
+        for i0 in starts:
+            work(i0)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(work, starts))
+    return out.reshape(x.shape)
 
 
 def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
-    """Widen bf16 bit patterns (uint16) to float32 exactly."""
+    """Widen bf16 bit patterns (uint16) to float32 exactly (block by block)."""
     b = np.ascontiguousarray(bits, dtype=np.uint16)
-    return (b.astype(np.uint32) << 16).view(np.float32)
+    flat = b.reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint32)
+    starts = range(0, flat.size, _ROUND_BLOCK)
+
+    def work(i0: int) -> None:
+        o = out[i0:i0 + _ROUND_BLOCK]
+        o[...] = flat[i0:i0 + _ROUND_BLOCK]
+        o <<= 16
+
+    if flat.size <= _ROUND_BLOCK:
+        for i0 in starts:
+            work(i0)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(work, starts))
+    return out.view(np.float32).reshape(b.shape)
 
 
 # ---------------------------------------------------------------------------

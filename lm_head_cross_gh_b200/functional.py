@@ -3,7 +3,7 @@
 
 Every loss is computed by the library's kernels in the forward call, together
 with its gradients (they come out of the same passes); ``backward`` returns
-them, scaled by the upstream gradient when that is not 1.  PyTorch only holds
+them, multiplied on the device by the upstream gradient.  PyTorch only holds
 the tensors: there is no other implementation behind these functions.
 
 * ``cross_entropy(logits, target, ignore_index, reduction, z_loss_multiplier)``
@@ -38,11 +38,13 @@ __all__ = ["cross_entropy", "chunked_linear_cross_entropy", "chunked_linear_loss
 
 
 def _scaled(grad, g):
-    """grad * g for a scalar upstream gradient g, without a pass when g == 1."""
+    """grad * g for the scalar upstream gradient g.
+
+    The product is always formed on the device: testing ``g == 1`` first would
+    read g back to the host, which stalls the stream on every backward and is
+    not allowed while a CUDA graph is being captured."""
     if grad is None:
         return None
-    if g.numel() == 1 and bool(g.reshape(()) == 1):
-        return grad
     return grad * g.to(grad.dtype)
 
 

@@ -22,8 +22,7 @@ Sources (the Greyhound functional API page, ``greyhound.nn.functional``):
 * nuvec ``FastOp::CrossEntropy`` / ``CrossEntropyVjp`` — the row loss
   definition and its logits gradient.
 
-Readings where the API documentation is silent (each is listed in the design
-notes):
+Readings where the API documentation is silent:
 z-loss is ``z * lse**2`` per valid token, added before the reduction; ``mean``
 with no valid token returns 0 with zero gradients; ``mean`` across chunks
 divides by the global valid-token count; a target equal to ``ignore_index`` is

@@ -3,14 +3,13 @@
 * `bench.py --impl reference` (the float64 oracle on host cores) prints one JSON
   line with the contract's keys, for the CE and the linear-CE workloads and for
   the forward-only operations.
-* Every summary under profiles/ gives the ncu command it came from; a summary
-  that states DRAM traffic also states the source digest and the workload, and
-  bench.py's parser reads it back.
+* Every summary under profiles/ gives the ncu command it came from; every DRAM
+  traffic figure bench.py reports comes from profiles/traffic.json, whose
+  entries are backed by a summary with the same figure, digest and workload.
 """
 import glob
 import json
 import os
-import re
 import subprocess
 import sys
 
@@ -48,17 +47,26 @@ def test_reference_arm_linear_ce_sample():
 
 
 def test_profile_summaries_state_their_command_and_source():
-    import bench
     files = sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md")))
     assert files
     for f in files:
         txt = open(f).read()
         assert "ncu " in txt, f"{f} does not give the ncu command"
-        if "traffic_bytes_per_launch" in txt:
-            assert re.search(r"source_sha:\s*[0-9a-f]{12}", txt), f
-            for m in re.finditer(r"workload:\s*(\S+)\s*\ntraffic_bytes_per_launch:\s*([0-9]+)", txt):
-                sha = re.search(r"source_sha:\s*([0-9a-f]+)", txt).group(1)
-                kernel = os.path.basename(f).split("_gpt2")[0].split("_fwd")[0]
-                kernel = kernel if kernel != "ce_ring_kernel" else "ce_ring_kernel_fwd"
-                got = bench.profiled_traffic(kernel, sha, m.group(1))
-                assert got == float(m.group(2)), (f, kernel, got)
+
+
+def test_traffic_entries_are_backed_by_a_summary_and_read_back():
+    """Every DRAM-traffic figure bench.py reports comes from profiles/traffic.json;
+    each entry names the summary that holds the same figure, its source digest
+    and its workload, and bench.profiled_traffic returns it for exactly that
+    (kernel, digest, workload)."""
+    import bench
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+        entries = json.load(fh)["entries"]
+    assert entries
+    for e in entries:
+        txt = open(os.path.join(ROOT, "profiles", e["summary"])).read()
+        assert str(e["traffic_bytes_per_launch"]) in txt, e
+        assert e["source_sha"] in txt and e["workload"] in txt, e
+        assert bench.profiled_traffic(e["kernel"], e["source_sha"], e["workload"]) == \
+            float(e["traffic_bytes_per_launch"])
+        assert bench.profiled_traffic(e["kernel"], "0" * 12, e["workload"]) is None

@@ -50,6 +50,32 @@ def test_cross_entropy_autograd_matches_the_kernel(cuda_device):
 
 
 @pytest.mark.gpu
+def test_backward_is_captured_in_a_cuda_graph(cuda_device):
+    """The backward multiplies the saved gradient by the upstream gradient on
+    the device, without reading it back to the host, so it can be captured in
+    a CUDA graph; each replay uses the upstream gradient's current value."""
+    p = gh_synth.ce_normal(300, 2003, 3.0, dtype="bf16", ignore_frac=0.1, z_loss=1e-4, seed=9)
+    x0 = torch.from_numpy(p.logits.view(np.int16)).cuda().view(torch.bfloat16)
+    t = torch.from_numpy(p.targets).cuda()
+    _, ref_grad = gh.gh_ce_fwd_bwd(x0, t, -100, "mean", 1e-4)
+    x = x0.clone().requires_grad_(True)
+    g = torch.full((), 2.0, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        loss = GF.cross_entropy(x, t, -100, "mean", 1e-4)
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        (gx,) = torch.autograd.grad(loss, x, grad_outputs=g, retain_graph=True)
+    for scale in (2.0, -0.5):
+        g.fill_(scale)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(gx, ref_grad * torch.tensor(scale, dtype=torch.bfloat16, device="cuda"))
+
+
+@pytest.mark.gpu
 def test_linear_and_generic_chunked_losses_autograd(cuda_device):
     q = gh_synth.linear_ce_normal(512, 128, 3001, chunk=0, ignore_frac=0.05, x_sigma=1.0, w_sigma=0.05,
                                   reduction="sum", z_loss=0.0, seed=4)

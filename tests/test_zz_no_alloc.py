@@ -23,6 +23,18 @@ from ce_check import check_grad, check_loss, grad_to_f64, loss_atol, row_eps, to
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=["auto", "rows", "ring"])
+def ce_path(request, monkeypatch):
+    """The row count picks the kernel (the two-pass ring from 8 rows per SM,
+    the row kernel below); "rows" and "ring" force one of them, so both
+    kernels run with the fixed scratch whatever the batch size."""
+    if request.param != "auto":
+        monkeypatch.setenv("GH_CE_PATH", request.param)
+    else:
+        monkeypatch.delenv("GH_CE_PATH", raising=False)
+    return request.param
+
+
 def _call_noalloc(x, t, p, loss, grad):
     L = gh.lib()
     dtype = gh.GH_F32 if x.dtype == torch.float32 else gh.GH_BF16
@@ -43,12 +55,15 @@ def _compare(p, loss_a, grad_a, loss_b, grad_b, what):
     check_grad(grad_b, grad_a, p.dtype, scale, p.targets, p.ignore_index, eps, what)
 
 
-def test_noalloc_matches_allocating_entry_point_on_two_calls_in_a_row(cuda_device):
-    # The second problem has a different row count, more ignored rows and the
-    # other reduction, so leftovers of the first call in the shared scratch
-    # (counter or row losses) would change its result.
+def test_noalloc_matches_allocating_entry_point_on_two_calls_in_a_row(cuda_device, ce_path):
+    # Each problem has a different row count, share of ignored rows or
+    # reduction than the one before it, so leftovers of the previous call in
+    # the shared scratch (counter or row losses) would change its result.  The
+    # 2048-row problem is past 8 rows per SM, where the library picks the ring
+    # kernel by itself.
     problems = [
         gh_synth.ce_normal(512, 50257, 3.0, dtype="bf16", ignore_frac=0.02, reduction="mean", z_loss=1e-4, seed=21),
+        gh_synth.ce_normal(2048, 4099, 3.0, dtype="bf16", ignore_frac=0.05, reduction="mean", z_loss=1e-4, seed=24),
         gh_synth.ce_normal(300, 4099, 2.0, dtype="f32", ignore_frac=0.30, reduction="mean", z_loss=0.0, seed=22),
         gh_synth.ce_normal(200, 50257, 3.0, dtype="bf16", ignore_frac=0.10, reduction="sum", z_loss=1e-4, seed=23),
     ]
