@@ -119,3 +119,30 @@ def test_full_size_llama3_8b_head_sampled(cuda_device):
     a, b = float(np.sum(dW * W)), float(np.sum(dX * X))
     assert abs(a - b) <= 2e-2 * max(abs(a), abs(b))
     assert np.isfinite(loss) and 0 < loss < 2 * np.log(p.V)
+
+
+@pytest.mark.parametrize("accum", ["weight", "fp32"])
+def test_weight_accumulation_order_golden(cuda_device, accum):
+    """The hand-derived two-chunk example of tests/golden/linear_ce_weight_accum.json,
+    bit for bit: 'weight' rounds the running bf16 sum after each chunk, 'fp32'
+    rounds once at the end.  D is padded from 2 to 8 with zero columns (the
+    library needs 16-byte rows); the padding columns' gradients are zero."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "linear_ce_weight_accum.json")) as f:
+        g = json.load(f)
+    X = np.zeros((g["N"], 8), np.float32)
+    X[:, :g["D"]] = np.array(g["inputs"], np.float32)
+    W = np.zeros((g["V"], 8), np.float32)
+    Xd = torch.from_numpy(X).cuda().to(torch.bfloat16)
+    Wd = torch.from_numpy(W).cuda().to(torch.bfloat16)
+    t = torch.tensor(g["targets"], dtype=torch.int64, device="cuda")
+    loss, dX, dW = gh.gh_linear_ce(Xd, Wd, t, g["ignore_index"], g["reduction"], g["z_loss"], g["chunk"], accum)
+    torch.cuda.synchronize()
+    key = "grad_weight_weight_accum_bf16_bits" if accum == "weight" else "grad_weight_fp32_accum_bf16_bits"
+    want = np.array([[int(b, 16) for b in row] for row in g[key]], dtype=np.uint16)
+    got = dW.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got[:, :g["D"]], want)
+    assert not got[:, g["D"]:].any()
+    assert not dX.float().cpu().numpy().any()
+    assert abs(loss.item() - 4 * np.log(2.0)) <= 1e-6

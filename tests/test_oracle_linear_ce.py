@@ -126,3 +126,35 @@ def test_zero_and_ignored_rows():
     t[:] = -100
     r = oracle.linear_cross_entropy(X, W, t, chunk=3)
     assert r["loss"] == 0.0 and not r["grad_inputs"].any() and not r["grad_weight"].any()
+
+
+def _golden_weight_accum():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "linear_ce_weight_accum.json")) as f:
+        return json.load(f)
+
+
+def _bits_to_f64(bits):
+    return np.array([[np.uint32(int(b, 16) << 16).view(np.float32) for b in row] for row in bits], dtype=np.float64)
+
+
+def test_weight_accumulation_order_golden():
+    """Hand-derived two-chunk example (tests/golden/linear_ce_weight_accum.json):
+    'weight' accumulation rounds the running sum after each chunk, which gives
+    different bits from rounding each chunk's product first and from a single
+    final rounding ('fp32')."""
+    g = _golden_weight_accum()
+    X = np.array(g["inputs"], dtype=np.float64)
+    W = np.array(g["weight"], dtype=np.float64)
+    t = np.array(g["targets"], dtype=np.int64)
+    w = oracle.linear_cross_entropy(X, W, t, g["ignore_index"], g["reduction"], g["z_loss"], g["chunk"], "weight")
+    f = oracle.linear_cross_entropy(X, W, t, g["ignore_index"], g["reduction"], g["z_loss"], g["chunk"], "fp32")
+    np.testing.assert_array_equal(w["grad_weight"], _bits_to_f64(g["grad_weight_weight_accum_bf16_bits"]))
+    np.testing.assert_array_equal(oracle.bf16_round(f["grad_weight"]),
+                                  _bits_to_f64(g["grad_weight_fp32_accum_bf16_bits"]))
+    assert not np.array_equal(w["grad_weight"], _bits_to_f64(g["wrong_reading_round_product_first_bits"]))
+    assert w["loss"] == pytest.approx(4 * np.log(2.0), rel=1e-15)
+    np.testing.assert_array_equal(w["grad_inputs"], np.array(g["grad_inputs"]))
+    # the inputs are the bf16 values the expressions name
+    np.testing.assert_array_equal(X, oracle.bf16_round(X))
