@@ -35,7 +35,8 @@ unchunked case reduces to).
 """
 from .ce import (bf16_round, cross_entropy, ce_rows, ce_vjp, n_valid_and_scale,
                  selective_log_softmax)
-from .linear_ce import linear_cross_entropy, linear_cross_entropy_materialised
+from .linear_ce import (grad_input_rows, grad_weight_rows, linear_cross_entropy,
+                        linear_cross_entropy_materialised, loss_from_lse, row_lse)
 
 __all__ = [
     "bf16_round",
@@ -46,4 +47,8 @@ __all__ = [
     "selective_log_softmax",
     "linear_cross_entropy",
     "linear_cross_entropy_materialised",
+    "row_lse",
+    "loss_from_lse",
+    "grad_input_rows",
+    "grad_weight_rows",
 ]

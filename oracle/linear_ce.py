@@ -77,3 +77,72 @@ def linear_cross_entropy_materialised(X: np.ndarray, W: np.ndarray, targets: np.
     G = r["grad"]
     return {"loss": r["loss"], "grad_inputs": G @ W, "grad_weight": G.T @ X,
             "lse": r["lse"], "n_valid": r["n_valid"]}
+
+
+# ---------------------------------------------------------------------------
+# Sampled outputs: the same definitions evaluated for chosen rows or chosen
+# vocabulary entries, for problems too large to materialise (the Llama-3-8B
+# head's logits are 16384 x 128256).  Every one equals the corresponding
+# slice of ``linear_cross_entropy`` with fp32 accumulation.
+# ---------------------------------------------------------------------------
+
+def row_lse(X: np.ndarray, W: np.ndarray, row_block: int = 256) -> np.ndarray:
+    """lse_i = log sum_v exp(X_i . W_v) for every row, the logits formed one
+    block of rows at a time (float64, host BLAS)."""
+    X = np.asarray(X, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    N = X.shape[0]
+    lse = np.empty(N)
+    for r0 in range(0, N, row_block):
+        Z = X[r0:r0 + row_block] @ W.T
+        m = Z.max(axis=1)
+        lse[r0:r0 + row_block] = m + np.log(np.exp(Z - m[:, None]).sum(axis=1))
+    return lse
+
+
+def loss_from_lse(X: np.ndarray, W: np.ndarray, targets: np.ndarray, lse: np.ndarray,
+                  ignore_index: int = -100, reduction: str = "mean", z_loss: float = 0.0) -> float:
+    """The reduced loss given every row's lse: row loss (lse - x_t) + z lse^2
+    for valid rows, x_t = X_i . W_{t_i}; summed, and divided by the valid
+    count for "mean"."""
+    X = np.asarray(X, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    t = np.asarray(targets, dtype=np.int64)
+    n_valid, _ = n_valid_and_scale(t, ignore_index, reduction, W.shape[0])
+    vr = np.nonzero(t != ignore_index)[0]
+    x_t = np.einsum("ij,ij->i", X[vr], W[t[vr]])
+    total = float(np.sum((lse[vr] - x_t) + z_loss * lse[vr] * lse[vr]))
+    return total / max(n_valid, 1) if reduction == "mean" else total
+
+
+def grad_input_rows(X: np.ndarray, W: np.ndarray, targets: np.ndarray, rows: np.ndarray,
+                    ignore_index: int = -100, reduction: str = "mean", z_loss: float = 0.0) -> np.ndarray:
+    """grad_inputs[rows] = G[rows] @ W, each row's logits gradient from its own
+    full logits row (the scale uses the valid count of all targets)."""
+    X = np.asarray(X, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    t = np.asarray(targets, dtype=np.int64)
+    _, scale = n_valid_and_scale(t, ignore_index, reduction, W.shape[0])
+    _, _, G = ce_rows(X[rows] @ W.T, t[rows], ignore_index, z_loss, scale)
+    return G @ W
+
+
+def grad_weight_rows(X: np.ndarray, W: np.ndarray, targets: np.ndarray, lse: np.ndarray,
+                     vocab: np.ndarray, ignore_index: int = -100, reduction: str = "mean",
+                     z_loss: float = 0.0) -> np.ndarray:
+    """grad_weight[vocab] = G[:, vocab]^T @ X (fp32 accumulation, unrounded):
+    the logits gradient's columns ``vocab``, by definition
+    G[i, v] = scale ((1 + 2 z lse_i) exp(X_i . W_v - lse_i) - [v == t_i]) for
+    valid rows and 0 for ignored rows, need only those columns of the logits
+    and every row's lse."""
+    X = np.asarray(X, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    t = np.asarray(targets, dtype=np.int64)
+    vocab = np.asarray(vocab, dtype=np.int64)
+    _, scale = n_valid_and_scale(t, ignore_index, reduction, W.shape[0])
+    valid = t != ignore_index
+    Zc = X @ W[vocab].T                                   # [N, len(vocab)]
+    G = (scale * (1.0 + 2.0 * z_loss * lse))[:, None] * np.exp(Zc - lse[:, None])
+    G -= scale * (valid[:, None] & (t[:, None] == vocab[None, :]))
+    G[~valid] = 0.0
+    return G.T @ X
