@@ -6,6 +6,12 @@
 //   dX_c     = G_c  W     A = G_c [rows, V]   K-major    B = W   [V, D]    N-major
 //   dW      += G_c^T X_c  A = G_c^T           M-major    B = X_c [rows, D] N-major
 //
+// For the cross-entropy the logits tile never leaves the chip as logits: the
+// epilogue (kEpiCeExp) turns each fp32 value into exp(x - R_row) and keeps the
+// row's sum and max over the tile, so the gradient GEMMs take G = diag(alpha) P
+// with P the stored exponentials (the row factor alpha is applied in the dX
+// epilogue as a row scale, and folded into X_c for dW).
+//
 // D[M, N] = sum_k A[m, k] B[n, k].  Tiles of 128 x kBN are computed by one CTA
 // (cta_group::1) in 64-wide K steps.  Warp roles:
 //   warp 0      TMA producer (one elected lane): A and B tiles into a ring of
@@ -48,7 +54,9 @@ enum GemmEpi : int {
   kEpiStoreBf16 = 0,  // out(bf16) = tile                       TMA store
   kEpiStoreF32 = 1,   // out(f32)  = tile                       TMA store
   kEpiAddF32 = 2,     // out(f32) += tile                       TMA reduce-add (in L2)
-  kEpiBf16Add = 3     // out = bf16(float(out) + tile), direct loads and stores (bf16 accumulator)
+  kEpiBf16Add = 3,    // out = bf16(float(out) + tile), direct loads and stores (bf16 accumulator)
+  kEpiCeExp = 4       // logits tile of the fused cross-entropy: out(bf16) = exp(tile - R_row)
+                      // (0 for ignored rows), plus per (row, column tile) sum and max
 };
 
 struct GemmArgs {
@@ -62,6 +70,17 @@ struct GemmArgs {
   void* out;            // kEpiBf16Add only: bf16 [M, ld_out]
   int64_t ld_out;
   int m_limit, n_limit; // kEpiBf16Add only: rows / columns stored (n_limit a multiple of 8)
+  // kEpiStoreBf16 / kEpiStoreF32: when non-null, output row r (of the M rows)
+  // is multiplied by row_scale[r] before it is stored.
+  const float* row_scale;
+  // kEpiCeExp: the logits tile of one chunk, M = chunk rows, N = V columns.
+  const int64_t* targets;  // [M] class ids; a row whose target is ignore_index or outside [0, N) is stored as 0
+  int64_t ignore_index;
+  float2* stats;           // [tiles_n][stats_ld]: (sum over the tile's columns of exp(x - R_row), max x)
+  int stats_ld;
+  float* x_target;         // [M]: the fp32 logit at the row's target column (valid rows)
+  const float* row_ref;    // [M] R_row, or null for R_row = 0
+  const int* run_flag;     // non-null: the kernel does nothing unless *run_flag != 0
 };
 
 // ---- PTX wrappers ----------------------------------------------------------------
@@ -193,7 +212,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_tiles = g.tiles_m * g.tiles_n * g.k_splits;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -220,6 +238,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_base_slot;
   pdl_wait();     // operands and outputs are free of the predecessor kernel from here on
   pdl_trigger();  // one CTA per SM, all resident: the next kernel may start its prologue
+  // A conditional launch whose flag is clear has no tile to compute (the flag
+  // was written by a kernel that completed before pdl_wait returned).
+  const int num_tiles_run = (g.run_flag && *reinterpret_cast<const volatile int*>(g.run_flag) == 0)
+                                ? 0
+                                : g.tiles_m * g.tiles_n * g.k_splits;
 
   // tile -> (m block, n block, K split); K splits vary slowest
   auto tile_coords = [&](int tile, int& mb, int& nb, int& ks) {
@@ -245,7 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool run = true;
-      for (int tile = blockIdx.x; tile < num_tiles && run; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < num_tiles_run && run; tile += gridDim.x) {
         int mb, nb, ks, kb0, kb1;
         tile_coords(tile, mb, nb, ks);
         kb_range(ks, kb0, kb1);
@@ -287,7 +310,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool run = true;
-      for (int tile = blockIdx.x; tile < num_tiles && run; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < num_tiles_run && run; tile += gridDim.x) {
         int mb, nb, ks, kb0, kb1;
         tile_coords(tile, mb, nb, ks);
         kb_range(ks, kb0, kb1);
@@ -331,14 +354,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     int nstore = 0;  // bulk groups committed by this warp (lane 0)
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < num_tiles_run; tile += gridDim.x) {
       int mb, nb, ks;
       tile_coords(tile, mb, nb, ks);
       if (!wait_or_abort(&tmem_full[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
       const int y = ks * g.split_rows + mb * kBM + q * 32;  // first output row of this warp
-      if (g.epi == kEpiStoreBf16) {
+      const int row = mb * kBM + q * 32 + lane;  // this thread's row of the M rows
+      if (g.epi == kEpiStoreBf16 || g.epi == kEpiCeExp) {
+        // kEpiCeExp: x -> exp(x - R) for valid rows (0 for ignored rows and the
+        // columns past N), with the row's sum and max over the tile's columns.
+        const bool ce = g.epi == kEpiCeExp;
+        float rs = 1.0f, nrl2 = 0.0f;
+        int tcol = -1;       // target column relative to the tile (-1: none)
+        bool keep = true;    // row stores its exponentials (valid row)
+        if (ce) {
+          keep = false;
+          if (row < g.M) {
+            const int64_t t = g.targets[row];
+            keep = t != g.ignore_index && t >= 0 && t < g.N;
+            if (keep && t >= static_cast<int64_t>(nb) * kBN && t < static_cast<int64_t>(nb) * kBN + kBN)
+              tcol = static_cast<int>(t - static_cast<int64_t>(nb) * kBN);
+            if (g.row_ref) nrl2 = -g.row_ref[row] * kLog2e;
+          }
+        } else if (g.row_scale) {
+          rs = row < g.M ? g.row_scale[row] : 0.0f;
+        }
+        const int cols_left = g.N - nb * kBN;  // columns of this tile inside N
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        float m0 = -INFINITY, m1 = -INFINITY;
         // 64-column slices: 2 TMEM loads -> 32 rows x 128 bytes, 128-byte swizzled
 #pragma unroll 1
         for (int cs = 0; cs < kBN; cs += 64) {
@@ -346,6 +391,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld32(t_row + cs, v0);
           tmem_ld32(t_row + cs + 32, v1);
           tmem_ld_wait();
+          if (ce) {
+            if (tcol >= cs && tcol < cs + 64) {
+              float xt = 0.f;
+#pragma unroll
+              for (int j = 0; j < 64; ++j)
+                if (j == tcol - cs) xt = __uint_as_float(j < 32 ? v0[j] : v1[j - 32]);
+              g.x_target[row] = xt;
+            }
+            const bool whole = cols_left >= cs + 64;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              uint32_t& w = j < 32 ? v0[j] : v1[j - 32];
+              const float x = __uint_as_float(w);
+              float e = 0.0f;
+              if (whole || cs + j < cols_left) {
+                e = ex2(fmaf(x, kLog2e, nrl2));
+                if (j & 1) m1 = fmaxf(m1, x); else m0 = fmaxf(m0, x);
+                switch (j & 3) {
+                  case 0: s0 += e; break;
+                  case 1: s1 += e; break;
+                  case 2: s2 += e; break;
+                  default: s3 += e; break;
+                }
+              }
+              w = __float_as_uint(keep ? e : 0.0f);
+            }
+          } else if (g.row_scale) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              v0[j] = __float_as_uint(__uint_as_float(v0[j]) * rs);
+              v1[j] = __float_as_uint(__uint_as_float(v1[j]) * rs);
+            }
+          }
           uint8_t* buf = my_stage + (nstore & 1) * kStageOutBytes;
           if (nstore >= 2) {
             if (lane == 0) bulk_wait_read_1();
@@ -370,13 +448,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           ++nstore;
         }
+        if (ce && row < g.M)
+          g.stats[static_cast<int64_t>(nb) * g.stats_ld + row] =
+              make_float2((s0 + s1) + (s2 + s3), fmaxf(m0, m1));
       } else if (g.epi == kEpiStoreF32 || g.epi == kEpiAddF32) {
         // 32-column slices: 1 TMEM load -> 32 rows x 128 bytes of fp32
+        const float rs = g.row_scale ? (row < g.M ? g.row_scale[row] : 0.0f) : 1.0f;
 #pragma unroll 1
         for (int cs = 0; cs < kBN; cs += 32) {
           uint32_t v[32];
           tmem_ld32(t_row + cs, v);
           tmem_ld_wait();
+          if (g.row_scale) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * rs);
+          }
           uint8_t* buf = my_stage + (nstore & 1) * kStageOutBytes;
           if (nstore >= 2) {
             if (lane == 0) bulk_wait_read_1();
@@ -398,7 +484,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else {
         // kEpiBf16Add: accumulate into the bf16 output with plain loads and stores
-        const int row = mb * kBM + q * 32 + lane;
         const bool row_ok = row < g.m_limit;
 #pragma unroll 1
         for (int cc = 0; cc < kBN; cc += 32) {

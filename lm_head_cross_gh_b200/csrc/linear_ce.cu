@@ -2,18 +2,34 @@
 // `chunked_linear_loss`): logits = X @ W^T are formed one row chunk at a time
 // and never materialised in full.  Per chunk c (rows [c0, c0 + rows)):
 //
-//   1  L      = X_c W^T               tcgen05 GEMM, bf16 chunk buffer [rows, ld]
-//   2  L     := G_c (in place)        the cross-entropy row kernel on the chunk:
-//                                     loss rows and the logits gradient, scaled
-//                                     by the valid-token count of the whole call
-//   3  dX_c   = G_c W                 tcgen05 GEMM (A K-major, B N-major)
-//   4  dW    (+)= G_c^T X_c           tcgen05 GEMM (both operands M/N-major);
+//   1  P      = exp(X_c W^T - R)      tcgen05 GEMM whose epilogue turns the fp32
+//                                     logits tile into bf16 exponentials P (0 for
+//                                     ignored rows) and keeps, per (row, 256-column
+//                                     tile), the sum of the exponentials, the max
+//                                     logit and the target logit (R = 0)
+//   2  finalize                       per row: lse, the row loss, the factor
+//                                     alpha = scale (1 + 2 z lse) exp(R - lse),
+//                                     the target element P[t] -= scale / alpha and
+//                                     Xs_c = bf16(alpha X_c); then the logits
+//                                     gradient is exactly G_c = diag(alpha) P
+//   3  (recompute)                    only when a row's lse fell outside
+//                                     [-40, 40], where exp(x) is not safe in
+//                                     fp32/bf16: steps 1 and 2 again with R = the
+//                                     row's max logit (both launches exit at once
+//                                     when no row asked for it)
+//   4  dX_c   = diag(alpha) (P W)     tcgen05 GEMM (A K-major, B N-major), the
+//                                     row factor applied in its epilogue
+//   5  dW    (+)= P^T Xs_c            tcgen05 GEMM (both operands M/N-major);
 //                                     fp32 accumulator across chunks (TMA store,
 //                                     then TMA reduce-add in L2), rounded once to
 //                                     bf16 at the end ("fp32"), or accumulated in
 //                                     the bf16 output ("weight")
 // When the dX tiles alone would leave SMs idle, dX splits K into fp32 partials
 // that a second kernel sums in a fixed order (deterministic).
+//
+// gh_chunked_linear_loss (a caller-provided loss per chunk) keeps the plain
+// form: step 1 stores the bf16 logits, the caller's callback overwrites them
+// with its gradient G_c, and steps 4-5 run with alpha = 1 and X_c.
 //
 // The loss is the fixed-order sum of all rows' losses, divided by the valid
 // count for "mean".  ld = round_up(V, 8) keeps chunk rows 16-byte aligned as
@@ -96,6 +112,110 @@ __global__ void cast_bf16_kernel(const float* __restrict__ acc, int64_t n4, uint
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float4 a = reinterpret_cast<const float4*>(acc)[i];
     reinterpret_cast<uint2*>(out)[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+}
+
+// Per-chunk step 2 of the fused cross-entropy (one CTA of 256 threads per 32
+// rows).  Each row's statistics are combined over the column tiles in a fixed
+// order (deterministic): S = sum of the tiles' sums of exp(x - R), M = max.
+struct FinalizeArgs {
+  const float2* stats;      // [tiles_n][stats_ld]
+  int stats_ld, tiles_n;
+  const int64_t* targets;   // chunk rows
+  int64_t ignore_index;
+  int V, rows, D;
+  float z;
+  int mean;
+  const unsigned long long* n_valid;
+  const float* x_target;    // [rows] fp32 target logits
+  float* row_max;           // [rows]: written by the first pass, the recompute's R
+  int recompute;            // 0: first pass (R = 0); 1: recompute (R = row_max)
+  int* flag;                // first pass: set when a row needs the recompute; recompute: runs only if set
+  float* alpha;             // [rows]
+  float* row_loss;          // [rows] (this chunk's slice)
+  uint16_t* P;              // [rows, ld] exponentials of the chunk
+  int64_t ld;
+  const uint16_t* X;        // [rows, D] inputs of the chunk
+  uint16_t* Xs;             // [rows, D] alpha-scaled inputs
+};
+
+// exp(x) with R = 0 is exact to fp32 rounding and neither overflows nor loses
+// the row to underflow while the row's lse stays within this window.
+constexpr float kLseWindow = 40.0f;
+// |1 + 2 z lse| is raised to at least this value, so scale / alpha stays finite;
+// the gradient entries this changes are below scale * 2^-20 (the bf16 rounding
+// of the target entry alone is scale * 2^-9).
+constexpr float kZFactorFloor = 9.5367431640625e-07f;  // 2^-20
+
+__global__ void __launch_bounds__(256) lce_finalize_kernel(FinalizeArgs a) {
+  __shared__ float sh_s[8][32];
+  __shared__ float sh_m[8][32];
+  __shared__ float sh_alpha[32];
+  pdl_wait();
+  pdl_trigger();
+  if (a.recompute && *reinterpret_cast<const volatile int*>(a.flag) == 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * 32;
+  const int row = row0 + lane;
+  float s = 0.0f, m = -INFINITY;
+  if (row < a.rows) {
+    for (int nb = warp; nb < a.tiles_n; nb += 8) {
+      const float2 v = a.stats[static_cast<int64_t>(nb) * a.stats_ld + row];
+      s += v.x;
+      m = fmaxf(m, v.y);
+    }
+  }
+  sh_s[warp][lane] = s;
+  sh_m[warp][lane] = m;
+  __syncthreads();
+  if (warp == 0) {
+    float alpha = 0.0f;
+    if (row < a.rows) {
+      float S = 0.0f, M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        S += sh_s[w][lane];
+        M = fmaxf(M, sh_m[w][lane]);
+      }
+      const int64_t t = a.targets[row];
+      const bool valid = t != a.ignore_index && t >= 0 && t < a.V;
+      const float R = a.recompute ? a.row_max[row] : 0.0f;
+      if (!a.recompute) a.row_max[row] = M;
+      float loss = 0.0f;
+      if (valid) {
+        const float lse = R + logf(S);
+        const bool ok = a.recompute || (lse >= -kLseWindow && lse <= kLseWindow);
+        if (!ok) {
+          atomicExch(a.flag, 1);  // this chunk runs the recompute; its outputs come from there
+        } else {
+          float f = fmaf(2.0f * a.z, lse, 1.0f);
+          if (!(fabsf(f) >= kZFactorFloor)) f = f < 0.0f ? -kZFactorFloor : kZFactorFloor;
+          const unsigned long long nv = *a.n_valid;
+          const float scale = a.mean ? 1.0f / static_cast<float>(nv > 0 ? nv : 1ull) : 1.0f;
+          const float xt = a.x_target[row];
+          alpha = scale * f * expf(R - lse);
+          loss = (lse - xt) + a.z * lse * lse;
+          // G[t] = alpha (exp(x_t - R) - scale / alpha) = scale ((1 + 2 z lse) p_t - 1)
+          a.P[static_cast<int64_t>(row) * a.ld + t] = to_bf16_bits(expf(xt - R) - scale / alpha);
+        }
+      }
+      a.row_loss[row] = loss;
+      a.alpha[row] = alpha;
+    }
+    sh_alpha[lane] = alpha;
+  }
+  __syncthreads();
+  // Xs = bf16(alpha X) for this block's rows, 16-byte vectors
+  const int d8 = a.D / 8;
+  const int nrows = min(32, a.rows - row0);
+  for (int i = threadIdx.x; i < nrows * d8; i += 256) {
+    const int r = i / d8, c = i - r * d8;
+    const int64_t off = static_cast<int64_t>(row0 + r) * a.D + 8 * c;
+    const uint4 x = *reinterpret_cast<const uint4*>(a.X + off);
+    const float al = sh_alpha[r];
+    *reinterpret_cast<uint4*>(a.Xs + off) =
+        make_uint4(pack_bf16x2(bf16_lo(x.x) * al, bf16_hi(x.x) * al), pack_bf16x2(bf16_lo(x.y) * al, bf16_hi(x.y) * al),
+                   pack_bf16x2(bf16_lo(x.z) * al, bf16_hi(x.z) * al), pack_bf16x2(bf16_lo(x.w) * al, bf16_hi(x.w) * al));
   }
 }
 
@@ -189,15 +309,31 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const int dx_splits = choose_splits(dx_tiles_max, dx_num_kb, sms);
   const int64_t rows_pad = static_cast<int64_t>(tiles_m_max) * sm100::kBM;
 
-  // scratch: [counter | row losses | chunk buffer | fp32 dW accumulator | dX split partials]
+  const bool custom = a.loss_fn != nullptr;
+  const bool fused = !custom;  // the cross-entropy in the logits GEMM's epilogue
+  const int tiles_n_logits = static_cast<int>((V + sm100::kBN - 1) / sm100::kBN);
+
+  // scratch: [counter | row losses | chunk buffer | fp32 dW accumulator | dX split partials |
+  //           fused only: tile statistics | target logits | row max | alpha | scaled inputs | flags]
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t off_rows = 256;
-  const size_t off_buf = (off_rows + sizeof(float) * N + 255) / 256 * 256;
+  const size_t off_buf = up(off_rows + sizeof(float) * N);
   const size_t buf_bytes = static_cast<size_t>(chunk) * ld * 2;
-  const size_t off_acc = (off_buf + buf_bytes + 255) / 256 * 256;
+  const size_t off_acc = up(off_buf + buf_bytes);
   const size_t acc_bytes = acc32 ? static_cast<size_t>(V) * D * 4 : 0;
-  const size_t off_ws = (off_acc + acc_bytes + 255) / 256 * 256;
+  const size_t off_ws = up(off_acc + acc_bytes);
   const size_t ws_bytes = dx_splits > 1 ? static_cast<size_t>(dx_splits) * rows_pad * D * 4 : 0;
-  const size_t total = off_ws + ws_bytes;
+  const size_t off_stats = up(off_ws + ws_bytes);
+  const size_t stats_bytes = fused ? static_cast<size_t>(tiles_n_logits) * rows_pad * sizeof(float2) : 0;
+  const size_t off_xt = up(off_stats + stats_bytes);
+  const size_t vec_bytes = fused ? static_cast<size_t>(rows_pad) * sizeof(float) : 0;
+  const size_t off_rmax = up(off_xt + vec_bytes);
+  const size_t off_alpha = up(off_rmax + vec_bytes);
+  const size_t off_xs = up(off_alpha + vec_bytes);
+  const size_t xs_bytes = fused ? static_cast<size_t>(rows_pad) * D * 2 : 0;
+  const size_t off_flags = up(off_xs + xs_bytes);
+  const size_t flags_bytes = fused ? static_cast<size_t>(nchunks) * sizeof(int) : 0;
+  const size_t total = off_flags + flags_bytes;
   void* scratch = nullptr;
   gh_status_t st = scratch_alloc(&scratch, total, stream);
   if (st != GH_OK) return st;
@@ -208,16 +344,22 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   uint16_t* L = reinterpret_cast<uint16_t*>(base + off_buf);
   float* acc = acc32 ? reinterpret_cast<float*>(base + off_acc) : nullptr;
   float* ws = dx_splits > 1 ? reinterpret_cast<float*>(base + off_ws) : nullptr;
+  float2* stats = fused ? reinterpret_cast<float2*>(base + off_stats) : nullptr;
+  float* x_target = fused ? reinterpret_cast<float*>(base + off_xt) : nullptr;
+  float* row_max = fused ? reinterpret_cast<float*>(base + off_rmax) : nullptr;
+  float* alpha = fused ? reinterpret_cast<float*>(base + off_alpha) : nullptr;
+  uint16_t* Xs = fused ? reinterpret_cast<uint16_t*>(base + off_xs) : nullptr;
+  int* flags = fused ? reinterpret_cast<int*>(base + off_flags) : nullptr;
 
   const uint16_t* X = static_cast<const uint16_t*>(a.X);
   const uint16_t* W = static_cast<const uint16_t*>(a.W);
   uint16_t* dX = static_cast<uint16_t*>(a.dX);
   uint16_t* dW = static_cast<uint16_t*>(a.dW);
 
-  const bool custom = a.loss_fn != nullptr;
   st = custom    ? (cudaMemsetAsync(a.loss, 0, sizeof(float), stream) == cudaSuccess ? GH_OK : GH_ERR_CUDA)
        : a.n_total ? GH_OK
                    : ce_count_launch(a.targets, N, V, a.ignore_index, counter, stream);
+  if (st == GH_OK && fused && cudaMemsetAsync(flags, 0, flags_bytes, stream) != cudaSuccess) st = GH_ERR_CUDA;
   // W as the K-major B operand of the logits GEMM and the N-major B operand of
   // dX; the weight-gradient output (bf16) and accumulator (fp32) maps.
   CUtensorMap tm_w_k, tm_w_n, tm_dw_out, tm_acc, tm_ws;
@@ -232,44 +374,87 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     const int rows = static_cast<int>(std::min<int64_t>(chunk, N - c0));
     const uint16_t* Xc = X + c0 * D;
 
+    // the B operand of dW: the chunk's inputs, scaled by alpha on the fused path
+    const uint16_t* Bdw = fused ? Xs : Xc;
     CUtensorMap tm_x_k, tm_l_k, tm_l_m, tm_x_n, tm_l_out, tm_dx_out;
     if (!make_tmap(&tm_x_k, Xc, D, rows, D * 2, sm100::kBM) || !make_tmap(&tm_l_k, L, V, rows, ld * 2, sm100::kBM) ||
-        !make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) || !make_tmap(&tm_x_n, Xc, D, rows, D * 2, 64) ||
+        !make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) || !make_tmap(&tm_x_n, Bdw, D, rows, D * 2, 64) ||
         !make_out_bf16(&tm_l_out, L, V, rows, ld) || !make_out_bf16(&tm_dx_out, dX + c0 * D, D, rows, D)) {
       st = GH_ERR_CUDA;
       break;
     }
 
-    // 1: L = X_c W^T
-    sm100::GemmArgs g1 = gemm_args(rows, static_cast<int>(V), static_cast<int>(D), 1, sm100::kEpiStoreBf16);
-    st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, GH_KERNEL_LOGITS_GEMM, stream);
-    if (st != GH_OK) break;
-
-    // 2: per-row loss and the logits gradient, in place (the caller's loss, or
-    // the cross-entropy row kernels)
-    if (custom) {
-      st = a.loss_fn(a.loss_ctx, c0, rows, L, ld, V, a.loss, stream);
+    if (fused) {
+      // 1: P = exp(X_c W^T) with the row statistics
+      sm100::GemmArgs g1 = gemm_args(rows, static_cast<int>(V), static_cast<int>(D), 1, sm100::kEpiCeExp);
+      g1.targets = a.targets + c0;
+      g1.ignore_index = a.ignore_index;
+      g1.stats = stats;
+      g1.stats_ld = static_cast<int>(rows_pad);
+      g1.x_target = x_target;
+      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, GH_KERNEL_LOGITS_GEMM, stream);
       if (st != GH_OK) break;
+      // 2: lse, loss, alpha, the target entries and the scaled inputs
+      FinalizeArgs fa{};
+      fa.stats = stats;
+      fa.stats_ld = static_cast<int>(rows_pad);
+      fa.tiles_n = tiles_n_logits;
+      fa.targets = a.targets + c0;
+      fa.ignore_index = a.ignore_index;
+      fa.V = static_cast<int>(V);
+      fa.rows = rows;
+      fa.D = static_cast<int>(D);
+      fa.z = a.z;
+      fa.mean = a.mean;
+      fa.n_valid = n_valid;
+      fa.x_target = x_target;
+      fa.row_max = row_max;
+      fa.flag = flags + c;
+      fa.alpha = alpha;
+      fa.row_loss = row_loss + c0;
+      fa.P = L;
+      fa.ld = ld;
+      fa.X = Xc;
+      fa.Xs = Xs;
+      const dim3 fgrid(static_cast<unsigned>((rows + 31) / 32));
+      {
+        ProfileScope prof(GH_KERNEL_CHUNK_CE, stream);
+        const cudaError_t e = launch_pdl(lce_finalize_kernel, fgrid, dim3(256), 0, stream, 1, fa);
+        note_launch();
+        if (e != cudaSuccess) {
+          st = GH_ERR_CUDA;
+          break;
+        }
+      }
+      // 3: the recompute with R = the row max, for a chunk whose flag the finalize set
+      sm100::GemmArgs g1r = g1;
+      g1r.row_ref = row_max;
+      g1r.run_flag = flags + c;
+      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1r, GH_KERNEL_CHUNK_CE, stream);
+      if (st != GH_OK) break;
+      fa.recompute = 1;
+      {
+        ProfileScope prof(GH_KERNEL_CHUNK_CE, stream);
+        const cudaError_t e = launch_pdl(lce_finalize_kernel, fgrid, dim3(256), 0, stream, 1, fa);
+        note_launch();
+        if (e != cudaSuccess) {
+          st = GH_ERR_CUDA;
+          break;
+        }
+      }
     } else {
-      CeArgs ca{};
-      ca.logits = L;
-      ca.grad = L;
-      ca.targets = a.targets + c0;
-      ca.V = V;
-      ca.ld = ld;
-      ca.ignore_index = a.ignore_index;
-      ca.z = a.z;
-      ca.mean = a.mean;
-      ca.n_valid = n_valid;
-      ca.row_loss = row_loss + c0;
-      ca.congruent = 1;
-      ca.profile_kind = GH_KERNEL_CHUNK_CE;
-      st = ce_launch(ca, rows, GH_BF16, stream);
+      // 1: L = X_c W^T
+      sm100::GemmArgs g1 = gemm_args(rows, static_cast<int>(V), static_cast<int>(D), 1, sm100::kEpiStoreBf16);
+      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, GH_KERNEL_LOGITS_GEMM, stream);
+      if (st != GH_OK) break;
+      // 2: the caller's loss and logits gradient, in place
+      st = a.loss_fn(a.loss_ctx, c0, rows, L, ld, V, a.loss, stream);
       if (st != GH_OK) break;
     }
 
     // 3: dX_c = G_c W (K split into fp32 partials when the tiles alone leave SMs idle)
     sm100::GemmArgs g3 = gemm_args(rows, static_cast<int>(D), static_cast<int>(V), 1, sm100::kEpiStoreBf16);
+    g3.row_scale = alpha;  // null on the plain path
     const int splits = choose_splits(g3.tiles_m * g3.tiles_n, g3.num_kb, sms);
     if (splits > 1 && ws) {
       g3.k_splits = std::min(splits, dx_splits);
