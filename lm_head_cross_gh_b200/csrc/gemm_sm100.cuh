@@ -12,18 +12,23 @@
 // with P the stored exponentials (the row factor alpha is applied in the dX
 // epilogue as a row scale, and folded into X_c for dW).
 //
-// D[M, N] = sum_k A[m, k] B[n, k].  Tiles of 128 x kBN are computed by one CTA
-// (cta_group::1) in 64-wide K steps.  Warp roles:
-//   warp 0      TMA producer (one elected lane): A and B tiles into a ring of
-//               kStages shared-memory stages, 128-byte swizzled
-//   warp 1      TMEM allocator and MMA issuer (one lane): 4 x tcgen05.mma
-//               (M=128, N=kBN, K=16) per stage, commits release stages and
-//               publish finished accumulators
+// D[M, N] = sum_k A[m, k] B[n, k], in 64-wide K steps, on tiles of 128 x 256
+// computed by one CTA (cta_group::1) or of 256 x 256 computed by a pair of CTAs
+// in a cluster (cta_group::2: each CTA loads its 128 A rows and 128 of the 256
+// B rows, the leader issues the MMAs, each CTA's TMEM holds its 128 rows).
+// Warp roles in each CTA:
+//   warp 0      TMA producer (one lane): A and B tiles into a ring of
+//               shared-memory stages, 128-byte swizzled; a pair's stage
+//               barrier lives in the leader and counts both CTAs' bytes
+//   warp 1      TMEM allocator; in the leader, the MMA issuer (one lane):
+//               4 x tcgen05.mma (K=16) per stage, commits release the stage
+//               (in both CTAs) and publish finished accumulators
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
 //               the 32 TMEM lanes its warp id selects), conversion, stores
-// Two accumulators of kBN fp32 columns (all 512 TMEM columns) let the
+// Two accumulators of 256 fp32 columns (all 512 TMEM columns) let the
 // epilogue of one tile overlap the MMAs of the next.  Every wait is bounded
-// (GH_ERR_TIMEOUT, then all roles stop and TMEM is freed).
+// (GH_ERR_TIMEOUT, then all roles stop, copies in flight land, the MMAs
+// finish and TMEM is freed).  No load is multicast.
 #pragma once
 
 #include <cuda.h>
@@ -34,18 +39,31 @@
 namespace gh {
 namespace sm100 {
 
-constexpr int kBM = 128;
-constexpr int kBN = 256;
+constexpr int kBM = 128;                      // accumulator rows of one CTA (TMEM lanes)
+constexpr int kBN = 256;                      // accumulator columns (one tcgen05.mma N)
 constexpr int kBK = 64;                       // one 128-byte swizzle row of bf16
-constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;        // 16 KiB
-constexpr int kBBytes = kBN * kBK * 2;        // 32 KiB
-constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 2 * kBN;            // two accumulators
 constexpr int kStageOutBytes = 4096;          // one epilogue staging buffer: 32 rows x 128 bytes
 constexpr int kOutBytes = 4 * 2 * kStageOutBytes;  // 4 epilogue warps x 2 buffers
-constexpr int kGemmSmem = 1024 /*align*/ + kStages * kStageBytes + kOutBytes + 256 /*barriers*/;
+
+// One CTA per tile (cta_group::1: 128 x 256 tiles, the CTA loads all 256 B
+// rows) or a CTA pair per tile (cta_group::2: 256 x 256 tiles, each CTA loads
+// its 128 A rows and 128 of the B rows, the leader issues the MMAs for both).
+// With half the B bytes per stage, the pair keeps 6 stages in flight where a
+// single CTA keeps 4, in the same shared memory.
+template <bool PAIR>
+struct GemmCfg {
+  static constexpr int kTileM = PAIR ? 2 * kBM : kBM;  // output rows of a tile
+  static constexpr int kBRows = PAIR ? kBN / 2 : kBN;  // B rows (N) this CTA loads per stage
+  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr int kBBytes = kBRows * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kSmem = 1024 /*align*/ + kStages * kStageBytes + kOutBytes + 256 /*barriers*/;
+};
+constexpr int kGemmSmem = GemmCfg<false>::kSmem;
+static_assert(GemmCfg<true>::kSmem <= 232448 && GemmCfg<false>::kSmem <= 232448, "shared memory per CTA");
 
 // Epilogue modes (what happens to the fp32 tile).  The first three go out
 // through the `tma_out` tensor map from a swizzled shared-memory staging
@@ -106,6 +124,16 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const 
                : "memory");
 }
 
+// tma_load_2d into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (`bar` a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(map), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
 // Allow at most one committed bulk group still reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -117,33 +145,70 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// TMEM allocation: cta_group::2 allocates the same columns in both CTAs of the
+// pair, issued by the same warp of each.
+template <bool PAIR>
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
+  if constexpr (PAIR)
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
 }
+template <bool PAIR>
 __device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  if constexpr (PAIR)
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  else
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
+template <bool PAIR>
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  if constexpr (PAIR)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
 // D(tmem) (+)= A(smem desc) x B(smem desc), bf16 inputs, fp32 accumulate.
+// cta_group::2: issued by the pair's leader; A rows and B rows come half from
+// each CTA's shared memory (same offsets), each CTA's TMEM receives its rows.
+template <bool PAIR>
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if constexpr (PAIR)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
-// Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread is done;
+// for a pair, on the barrier at the same offset in both CTAs (a commit, not a
+// load: no data moves between the CTAs).
+template <bool PAIR>
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+  if constexpr (PAIR)
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
@@ -177,14 +242,32 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool a_mn, bool 
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// One potentially blocking test of phase `parity`, acquiring at cluster scope
+// (arrivals may come from the other CTA of a pair).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait with an abort flag shared by all roles: returns false once any role
 // timed out (and records GH_ERR_TIMEOUT when this wait is the one that did).
+template <bool PAIR = false>
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity, 20000u)) return true;
+  auto test = [&]() {
+    return PAIR ? mbar_try_wait_cluster(a, parity, 20000u) : mbar_try_wait(a, parity, 20000u);
+  };
+  if (test()) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(a, parity, 20000u)) return true;
+    if (test()) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitTimeoutNs) {
       *abort_flag = 1;
@@ -194,12 +277,21 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   }
 }
 
+// Sleep for about `ns` nanoseconds (bounded by the global timer).
+__device__ __forceinline__ void sleep_ns_bounded(uint64_t ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 < ns) __nanosleep(1000);
+}
+
 // ---- the kernel --------------------------------------------------------------------
 
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                      const __grid_constant__ CUtensorMap tma_out, GemmArgs g) {
+  using C = GemmCfg<PAIR>;
+  constexpr int kStages = C::kStages;
+  constexpr int kStageBytes = C::kStageBytes;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
@@ -208,10 +300,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* empty = full + kStages;
   uint64_t* tmem_full = empty + kStages;
   uint64_t* tmem_empty = tmem_full + 2;
-  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
+  uint64_t* mma_done = tmem_empty + 2;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // A pair is a cluster of two consecutive CTAs; rank 0 (the leader) issues
+  // the MMAs, and its stage and accumulator barriers count both CTAs.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -220,8 +319,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], 128);
+      mbar_init(&tmem_empty[b], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
     }
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tma_a);
@@ -229,11 +329,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (g.epi != kEpiBf16Add) prefetch_tmap(&tma_out);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_base_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<PAIR>(tmem_base_slot, kTmemCols);
+    tmem_relinquish<PAIR>();
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {  // both CTAs' barriers are initialised before either signals the other
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
   pdl_wait();     // operands and outputs are free of the predecessor kernel from here on
@@ -263,62 +367,89 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   };
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs of a pair: each loads its halves) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t issued = 0;  // stages this producer armed
       bool run = true;
-      for (int tile = blockIdx.x; tile < num_tiles_run && run; tile += gridDim.x) {
+      for (int tile = unit; tile < num_tiles_run && run; tile += units) {
         int mb, nb, ks, kb0, kb1;
         tile_coords(tile, mb, nb, ks);
         kb_range(ks, kb0, kb1);
-        const int m0 = mb * kBM, n0 = nb * kBN;
+        const int m0 = mb * C::kTileM + static_cast<int>(rank) * kBM;
+        const int n0 = nb * kBN + static_cast<int>(rank) * C::kBRows;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!wait_or_abort(&empty[stage], phase ^ 1, abort_flag)) {
+          if (!wait_or_abort<PAIR>(&empty[stage], phase ^ 1, abort_flag)) {
             run = false;
             break;
           }
           uint8_t* sa = stage_base + stage * kStageBytes;
           uint8_t* sb = sa + kABytes;
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
           const int k0 = kb * kBK;
+          auto load = [&](void* dst, const CUtensorMap* map, int x, int y) {
+            if constexpr (PAIR) {
+              if (!leader) {
+                tma_load_2d_pair(dst, map, map_to_rank(&full[stage], 0), x, y);
+                return;
+              }
+            }
+            tma_load_2d(dst, map, &full[stage], x, y);
+          };
+          // the leader's stage barrier counts both CTAs' bytes
+          if (leader) mbar_arrive_expect_tx(&full[stage], PAIR ? 2 * kStageBytes : kStageBytes);
           if constexpr (A_MN) {
-            tma_load_2d(sa, &tma_a, &full[stage], m0, k0);
-            tma_load_2d(sa + 8192, &tma_a, &full[stage], m0 + 64, k0);
+            load(sa, &tma_a, m0, k0);
+            load(sa + 8192, &tma_a, m0 + 64, k0);
           } else {
-            tma_load_2d(sa, &tma_a, &full[stage], k0, m0);
+            load(sa, &tma_a, k0, m0);
           }
           if constexpr (B_MN) {
 #pragma unroll
-            for (int j = 0; j < kBN / 64; ++j) tma_load_2d(sb + j * 8192, &tma_b, &full[stage], n0 + 64 * j, k0);
+            for (int j = 0; j < C::kBRows / 64; ++j) load(sb + j * 8192, &tma_b, n0 + 64 * j, k0);
           } else {
-            tma_load_2d(sb, &tma_b, &full[stage], k0, n0);
+            load(sb, &tma_b, k0, n0);
           }
+          ++issued;
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
+      if (*abort_flag) {
+        // copies still in flight land before the CTA exits: the leader's stage
+        // barriers count them (both CTAs' for a pair); a pair's other CTA
+        // cannot see its own and waits out a fixed, generous interval instead
+        if (leader) {
+          const uint64_t t0 = global_timer_ns();
+          for (uint32_t n = (issued > kStages ? issued - kStages : 0); n < issued; ++n) {
+            const uint32_t a = smem_u32(&full[n % kStages]);
+            while (!mbar_try_wait(a, (n / kStages) & 1, 20000u) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+            }
+          }
+        }
+        if (PAIR) sleep_ns_bounded(200000);
+      }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc(kBM, kBN, A_MN, B_MN);
+    // ---------------- MMA issuer (the leader of a pair) ----------------
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = instr_desc(C::kTileM, kBN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool run = true;
-      for (int tile = blockIdx.x; tile < num_tiles_run && run; tile += gridDim.x) {
+      for (int tile = unit; tile < num_tiles_run && run; tile += units) {
         int mb, nb, ks, kb0, kb1;
         tile_coords(tile, mb, nb, ks);
         kb_range(ks, kb0, kb1);
-        if (!wait_or_abort(&tmem_empty[acc], acc_phase ^ 1, abort_flag)) break;
+        if (!wait_or_abort<PAIR>(&tmem_empty[acc], acc_phase ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!wait_or_abort(&full[stage], phase, abort_flag)) {
+          if (!wait_or_abort<PAIR>(&full[stage], phase, abort_flag)) {
             run = false;
             break;
           }
@@ -331,21 +462,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // M/N-major: it moves 16 rows (2 x 1024-byte swizzle atoms).
             const uint64_t ad = A_MN ? smem_desc(sa + k * 2048, 8192, 1024) : smem_desc(sa + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+            umma_bf16<PAIR>(d_tmem, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);  // stage free once these MMAs have read it
+          umma_commit<PAIR>(&empty[stage]);  // stage free (in both CTAs) once these MMAs have read it
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!run) break;
-        umma_commit(&tmem_full[acc]);  // accumulator complete
+        umma_commit<PAIR>(&tmem_full[acc]);  // accumulator complete
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
+      // every MMA issued has finished reading shared memory (both CTAs') and
+      // writing TMEM before the teardown
+      umma_commit<PAIR>(mma_done);
+      (void)mbar_wait(mma_done, 0);
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
@@ -354,14 +489,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     int nstore = 0;  // bulk groups committed by this warp (lane 0)
-    for (int tile = blockIdx.x; tile < num_tiles_run; tile += gridDim.x) {
+    for (int tile = unit; tile < num_tiles_run; tile += units) {
       int mb, nb, ks;
       tile_coords(tile, mb, nb, ks);
-      if (!wait_or_abort(&tmem_full[acc], acc_phase, abort_flag)) break;
+      if (!wait_or_abort<PAIR>(&tmem_full[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
-      const int y = ks * g.split_rows + mb * kBM + q * 32;  // first output row of this warp
-      const int row = mb * kBM + q * 32 + lane;  // this thread's row of the M rows
+      const int rbase = mb * C::kTileM + static_cast<int>(rank) * kBM + q * 32;  // this warp's first row
+      const int y = ks * g.split_rows + rbase;                                   // its first output row
+      const int row = rbase + lane;  // this thread's row of the M rows
       if (g.epi == kEpiStoreBf16 || g.epi == kEpiCeExp) {
         // kEpiCeExp: x -> exp(x - R) for valid rows (0 for ignored rows and the
         // columns past N), with the row's sum and max over the tile's columns.
@@ -510,9 +646,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      // every TMEM load of this accumulator is complete: hand it back to the MMA warp
+      // every TMEM load of this accumulator is complete: hand it back to the MMA
+      // warp (of the pair's leader)
       tc_fence_before();
-      mbar_arrive(&tmem_empty[acc]);
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(&tmem_empty[acc], 0));
+        else mbar_arrive(&tmem_empty[acc]);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -525,9 +666,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {  // neither CTA leaves while the other may still signal it or read its tiles
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc<PAIR>(tmem_base, kTmemCols);
   }
 }
 

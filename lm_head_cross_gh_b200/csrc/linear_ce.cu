@@ -37,6 +37,7 @@
 // never used.
 #include <algorithm>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "ce.h"
@@ -226,27 +227,46 @@ int sm_count() {
   return n;
 }
 
+// Tiles of the three GEMMs go to CTA pairs (cta_group::2, 256 x 256 tiles) by
+// default; GH_GEMM=single selects one CTA per 128 x 256 tile (tests,
+// measurements).
+bool use_pairs() {
+  const char* e = std::getenv("GH_GEMM");
+  return !(e && std::strcmp(e, "single") == 0);
+}
+
 template <bool A_MN, bool B_MN>
 gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
-                        const sm100::GemmArgs& g, int kind, cudaStream_t stream) {
-  auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN>;
-  if (ensure_smem_limit(kern, sm100::kGemmSmem) != cudaSuccess) return GH_ERR_CUDA;
+                        const sm100::GemmArgs& g, bool pair, int kind, cudaStream_t stream) {
   const int tiles = g.tiles_m * g.tiles_n * g.k_splits;
   if (tiles == 0) return GH_OK;
-  const int grid = std::min(tiles, sm_count());
-  ProfileScope prof(kind, stream);
-  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(sm100::kGemmThreads), sm100::kGemmSmem, stream, 1, ta, tb,
-                                   tout, g);
+  cudaError_t e;
+  if (pair) {
+    auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN, true>;
+    if (ensure_smem_limit(kern, sm100::GemmCfg<true>::kSmem) != cudaSuccess) return GH_ERR_CUDA;
+    const int pairs = std::min(tiles, std::max(1, sm_count() / 2));
+    ProfileScope prof(kind, stream);
+    e = launch_pdl(kern, dim3(2 * pairs), dim3(sm100::kGemmThreads), sm100::GemmCfg<true>::kSmem, stream, 2, ta, tb,
+                   tout, g);
+  } else {
+    auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN, false>;
+    if (ensure_smem_limit(kern, sm100::GemmCfg<false>::kSmem) != cudaSuccess) return GH_ERR_CUDA;
+    const int grid = std::min(tiles, sm_count());
+    ProfileScope prof(kind, stream);
+    e = launch_pdl(kern, dim3(grid), dim3(sm100::kGemmThreads), sm100::GemmCfg<false>::kSmem, stream, 1, ta, tb,
+                   tout, g);
+  }
   note_launch();
   return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
 }
 
-sm100::GemmArgs gemm_args(int M, int N, int K, int m_fastest, int epi) {
+sm100::GemmArgs gemm_args(int M, int N, int K, int m_fastest, int epi, bool pair) {
+  const int tile_m = pair ? sm100::GemmCfg<true>::kTileM : sm100::GemmCfg<false>::kTileM;
   sm100::GemmArgs g{};
   g.M = M;
   g.N = N;
   g.K = K;
-  g.tiles_m = (M + sm100::kBM - 1) / sm100::kBM;
+  g.tiles_m = (M + tile_m - 1) / tile_m;
   g.tiles_n = (N + sm100::kBN - 1) / sm100::kBN;
   g.num_kb = (K + sm100::kBK - 1) / sm100::kBK;
   g.k_splits = 1;
@@ -302,12 +322,15 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const int64_t nchunks = (N + chunk - 1) / chunk;
   if (chunk > INT32_MAX / 2 || V > INT32_MAX / 2) return GH_ERR_UNSUPPORTED;
   const bool acc32 = a.accum == GH_ACCUM_FP32 && nchunks > 1;
+  const bool pair = use_pairs();
+  const int tile_m = pair ? sm100::GemmCfg<true>::kTileM : sm100::GemmCfg<false>::kTileM;
   const int sms = sm_count();
-  const int tiles_m_max = static_cast<int>((chunk + sm100::kBM - 1) / sm100::kBM);
+  const int units = pair ? std::max(1, sms / 2) : sms;  // tile-processing units (CTA pairs or CTAs)
+  const int tiles_m_max = static_cast<int>((chunk + tile_m - 1) / tile_m);
   const int dx_num_kb = static_cast<int>((V + sm100::kBK - 1) / sm100::kBK);
   const int dx_tiles_max = tiles_m_max * static_cast<int>((D + sm100::kBN - 1) / sm100::kBN);
-  const int dx_splits = choose_splits(dx_tiles_max, dx_num_kb, sms);
-  const int64_t rows_pad = static_cast<int64_t>(tiles_m_max) * sm100::kBM;
+  const int dx_splits = choose_splits(dx_tiles_max, dx_num_kb, units);
+  const int64_t rows_pad = static_cast<int64_t>(tiles_m_max) * tile_m;
 
   const bool custom = a.loss_fn != nullptr;
   const bool fused = !custom;  // the cross-entropy in the logits GEMM's epilogue
@@ -364,7 +387,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   // dX; the weight-gradient output (bf16) and accumulator (fp32) maps.
   CUtensorMap tm_w_k, tm_w_n, tm_dw_out, tm_acc, tm_ws;
   if (st == GH_OK &&
-      (!make_tmap(&tm_w_k, W, D, V, D * 2, sm100::kBN) || !make_tmap(&tm_w_n, W, D, V, D * 2, 64) ||
+      (!make_tmap(&tm_w_k, W, D, V, D * 2, pair ? sm100::GemmCfg<true>::kBRows : sm100::GemmCfg<false>::kBRows) || !make_tmap(&tm_w_n, W, D, V, D * 2, 64) ||
        !make_out_bf16(&tm_dw_out, dW, D, V, D) || (acc32 && !make_out_f32(&tm_acc, acc, D, V, D)) ||
        (ws && !make_out_f32(&tm_ws, ws, D, dx_splits * rows_pad, D))))
     st = GH_ERR_CUDA;
@@ -386,13 +409,13 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
 
     if (fused) {
       // 1: P = exp(X_c W^T) with the row statistics
-      sm100::GemmArgs g1 = gemm_args(rows, static_cast<int>(V), static_cast<int>(D), 1, sm100::kEpiCeExp);
+      sm100::GemmArgs g1 = gemm_args(rows, static_cast<int>(V), static_cast<int>(D), 1, sm100::kEpiCeExp, pair);
       g1.targets = a.targets + c0;
       g1.ignore_index = a.ignore_index;
       g1.stats = stats;
       g1.stats_ld = static_cast<int>(rows_pad);
       g1.x_target = x_target;
-      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, GH_KERNEL_LOGITS_GEMM, stream);
+      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, pair, GH_KERNEL_LOGITS_GEMM, stream);
       if (st != GH_OK) break;
       // 2: lse, loss, alpha, the target entries and the scaled inputs
       FinalizeArgs fa{};
@@ -430,7 +453,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       sm100::GemmArgs g1r = g1;
       g1r.row_ref = row_max;
       g1r.run_flag = flags + c;
-      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1r, GH_KERNEL_CHUNK_CE, stream);
+      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1r, pair, GH_KERNEL_CHUNK_CE, stream);
       if (st != GH_OK) break;
       fa.recompute = 1;
       {
@@ -444,8 +467,8 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       }
     } else {
       // 1: L = X_c W^T
-      sm100::GemmArgs g1 = gemm_args(rows, static_cast<int>(V), static_cast<int>(D), 1, sm100::kEpiStoreBf16);
-      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, GH_KERNEL_LOGITS_GEMM, stream);
+      sm100::GemmArgs g1 = gemm_args(rows, static_cast<int>(V), static_cast<int>(D), 1, sm100::kEpiStoreBf16, pair);
+      st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, pair, GH_KERNEL_LOGITS_GEMM, stream);
       if (st != GH_OK) break;
       // 2: the caller's loss and logits gradient, in place
       st = a.loss_fn(a.loss_ctx, c0, rows, L, ld, V, a.loss, stream);
@@ -453,16 +476,16 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     }
 
     // 3: dX_c = G_c W (K split into fp32 partials when the tiles alone leave SMs idle)
-    sm100::GemmArgs g3 = gemm_args(rows, static_cast<int>(D), static_cast<int>(V), 1, sm100::kEpiStoreBf16);
+    sm100::GemmArgs g3 = gemm_args(rows, static_cast<int>(D), static_cast<int>(V), 1, sm100::kEpiStoreBf16, pair);
     g3.row_scale = alpha;  // null on the plain path
-    const int splits = choose_splits(g3.tiles_m * g3.tiles_n, g3.num_kb, sms);
+    const int splits = choose_splits(g3.tiles_m * g3.tiles_n, g3.num_kb, units);
     if (splits > 1 && ws) {
       g3.k_splits = std::min(splits, dx_splits);
       g3.kb_per_split = (g3.num_kb + g3.k_splits - 1) / g3.k_splits;
       g3.k_splits = (g3.num_kb + g3.kb_per_split - 1) / g3.kb_per_split;
       g3.split_rows = static_cast<int>(rows_pad);
       g3.epi = sm100::kEpiStoreF32;
-      st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_ws, g3, GH_KERNEL_DX_GEMM, stream);
+      st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_ws, g3, pair, GH_KERNEL_DX_GEMM, stream);
       if (st != GH_OK) break;
       const cudaError_t e = launch_pdl(splitk_reduce_kernel, dim3(sms * 4), dim3(256), 0, stream, 1,
                                        static_cast<const float*>(ws), g3.k_splits, rows_pad * D, rows,
@@ -473,12 +496,12 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
         break;
       }
     } else {
-      st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_dx_out, g3, GH_KERNEL_DX_GEMM, stream);
+      st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_dx_out, g3, pair, GH_KERNEL_DX_GEMM, stream);
       if (st != GH_OK) break;
     }
 
     // 4: dW (+)= G_c^T X_c
-    sm100::GemmArgs g4 = gemm_args(static_cast<int>(V), static_cast<int>(D), rows, 0, sm100::kEpiStoreBf16);
+    sm100::GemmArgs g4 = gemm_args(static_cast<int>(V), static_cast<int>(D), rows, 0, sm100::kEpiStoreBf16, pair);
     g4.out = dW;
     g4.ld_out = D;
     const CUtensorMap* out4 = &tm_dw_out;
@@ -490,7 +513,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     } else {
       g4.epi = c == 0 ? sm100::kEpiStoreBf16 : sm100::kEpiBf16Add;
     }
-    st = launch_gemm<true, true>(tm_l_m, tm_x_n, *out4, g4, GH_KERNEL_DW_GEMM, stream);
+    st = launch_gemm<true, true>(tm_l_m, tm_x_n, *out4, g4, pair, GH_KERNEL_DW_GEMM, stream);
   }
   if (st == GH_OK && acc32) {
     // the fp32 accumulator's single rounding to the weight dtype

@@ -1,4 +1,5 @@
-"""GPU parity of gh_linear_ce (chunked linear cross-entropy) against the oracle.
+"""GPU parity of gh_linear_ce (chunked linear cross-entropy) against the oracle,
+on both GEMM layouts (CTA pairs and single CTAs).
 
 Tolerances: the stated bars are loss within 1e-3 relative and grad_inputs /
 grad_weight within 1e-2 relative Frobenius error (bf16 GEMMs).  The GPU rounds
@@ -17,6 +18,14 @@ import lm_head_cross_gh_b200 as gh
 import oracle
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, params=["pair", "single"])
+def gemm_mode(request, monkeypatch):
+    """Every case on both GEMM layouts: 256 x 256 tiles on a pair of CTAs
+    (cta_group::2, the default) and 128 x 256 tiles on one CTA."""
+    monkeypatch.setenv("GH_GEMM", request.param)
+    return request.param
 
 
 def dev_bf16(a):
