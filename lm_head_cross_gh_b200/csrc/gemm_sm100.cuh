@@ -226,6 +226,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// tcgen05.wait::ld that also names the registers the loads fill, so no read
+// of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&a)[32], uint32_t (&b)[32]) {
+  tmem_ld_wait(a);
+  tmem_ld_wait(b);  // returns at once: the first wait covered every earlier load
+}
+
 // Shared-memory matrix descriptor (tcgen05): start address, leading and
 // stride byte offsets (all >> 4), version 1, base offset 0, 128-byte swizzle.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -498,9 +515,96 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int rbase = mb * C::kTileM + static_cast<int>(rank) * kBM + q * 32;  // this warp's first row
       const int y = ks * g.split_rows + rbase;                                   // its first output row
       const int row = rbase + lane;  // this thread's row of the M rows
-      if (g.epi == kEpiStoreBf16 || g.epi == kEpiCeExp) {
-        // kEpiCeExp: x -> exp(x - R) for valid rows (0 for ignored rows and the
-        // columns past N), with the row's sum and max over the tile's columns.
+      // 32 rows x 64 bf16 (this warp's slice at column x) to global memory
+      // through a 128-byte swizzled staging buffer and one TMA store.
+      auto store_slice = [&](const uint32_t (&pk)[32], int x) {
+        uint8_t* buf = my_stage + (nstore & 1) * kStageOutBytes;
+        if (nstore >= 2) {
+          if (lane == 0) bulk_wait_read_1();
+          __syncwarp();
+        }
+        uint8_t* rowp = buf + lane * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tma_out, buf, x, y);
+          bulk_commit();
+        }
+        ++nstore;
+      };
+      if (g.epi == kEpiCeExp && g.N - nb * kBN >= kBN) {
+        // A whole tile of the fused cross-entropy: every column is inside N.
+        // exp(x - R) = 2^(x log2 e - R log2 e) with packed f32x2 arithmetic; a
+        // reference of -inf stores 0 for rows that are ignored or past M.
+        float nr = -INFINITY;
+        int tcol = -1;
+        if (row < g.M) {
+          const int64_t t = g.targets[row];
+          if (t != g.ignore_index && t >= 0 && t < g.N) {
+            nr = g.row_ref ? -g.row_ref[row] * kLog2e : 0.0f;
+            const int64_t off = t - static_cast<int64_t>(nb) * kBN;
+            if (off >= 0 && off < kBN) tcol = static_cast<int>(off);
+          }
+        }
+        const float2 l2 = make_float2(kLog2e, kLog2e), n2 = make_float2(nr, nr);
+        float2 sA = make_float2(0.f, 0.f), sB = make_float2(0.f, 0.f);
+        float mA = -INFINITY, mB = -INFINITY;
+        auto slice = [&](const uint32_t (&u0)[32], const uint32_t (&u1)[32], int cs) {
+          if (tcol >= cs && tcol < cs + 64) {
+            float xt = 0.f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+              if (j == tcol - cs) xt = __uint_as_float(j < 32 ? u0[j] : u1[j - 32]);
+            g.x_target[row] = xt;
+          }
+          uint32_t pk[32];
+#pragma unroll
+          for (int j = 0; j < 64; j += 4) {
+            const uint32_t* u = j < 32 ? u0 : u1;
+            const int i = j & 31;
+            const float2 xa = make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1]));
+            const float2 xb = make_float2(__uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]));
+            const float2 ya = __ffma2_rn(xa, l2, n2);
+            const float2 yb = __ffma2_rn(xb, l2, n2);
+            const float2 ea = make_float2(ex2(ya.x), ex2(ya.y));
+            const float2 eb = make_float2(ex2(yb.x), ex2(yb.y));
+            sA = __fadd2_rn(sA, ea);
+            sB = __fadd2_rn(sB, eb);
+            mA = fmaxf(mA, fmaxf(xa.x, xa.y));
+            mB = fmaxf(mB, fmaxf(xb.x, xb.y));
+            pk[j / 2] = pack_bf16x2(ea.x, ea.y);
+            pk[j / 2 + 1] = pack_bf16x2(eb.x, eb.y);
+          }
+          store_slice(pk, nb * kBN + cs);
+        };
+        // two register sets: one slice's TMEM loads fly while the other is processed
+        uint32_t a0[32], a1[32], b0[32], b1[32];
+        tmem_ld32(t_row, a0);
+        tmem_ld32(t_row + 32, a1);
+        tmem_ld_wait(a0, a1);
+        tmem_ld32(t_row + 64, b0);
+        tmem_ld32(t_row + 96, b1);
+        slice(a0, a1, 0);
+        tmem_ld_wait(b0, b1);
+        tmem_ld32(t_row + 128, a0);
+        tmem_ld32(t_row + 160, a1);
+        slice(b0, b1, 64);
+        tmem_ld_wait(a0, a1);
+        tmem_ld32(t_row + 192, b0);
+        tmem_ld32(t_row + 224, b1);
+        slice(a0, a1, 128);
+        tmem_ld_wait(b0, b1);
+        slice(b0, b1, 192);
+        if (row < g.M)
+          g.stats[static_cast<int64_t>(nb) * g.stats_ld + row] =
+              make_float2((sA.x + sA.y) + (sB.x + sB.y), fmaxf(mA, mB));
+      } else if (g.epi == kEpiStoreBf16 || g.epi == kEpiCeExp) {
+        // The bf16 store (optionally row-scaled), and the fused cross-entropy's
+        // last column tile, whose columns past N are left out of the sum and max.
         const bool ce = g.epi == kEpiCeExp;
         float rs = 1.0f, nrl2 = 0.0f;
         int tcol = -1;       // target column relative to the tile (-1: none)
@@ -520,13 +624,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int cols_left = g.N - nb * kBN;  // columns of this tile inside N
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
         float m0 = -INFINITY, m1 = -INFINITY;
-        // 64-column slices: 2 TMEM loads -> 32 rows x 128 bytes, 128-byte swizzled
+        // 64-column slices: 2 TMEM loads -> 32 rows x 128 bytes, 128-byte swizzled.
+        // The next slice's TMEM loads are in flight while this one is processed.
+        uint32_t n0[32], n1[32];
+        tmem_ld32(t_row, n0);
+        tmem_ld32(t_row + 32, n1);
+        tmem_ld_wait(n0, n1);
 #pragma unroll 1
         for (int cs = 0; cs < kBN; cs += 64) {
           uint32_t v0[32], v1[32];
-          tmem_ld32(t_row + cs, v0);
-          tmem_ld32(t_row + cs + 32, v1);
-          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            v0[j] = n0[j];
+            v1[j] = n1[j];
+          }
+          if (cs + 64 < kBN) {
+            tmem_ld32(t_row + cs + 64, n0);
+            tmem_ld32(t_row + cs + 96, n1);
+          }
           if (ce) {
             if (tcol >= cs && tcol < cs + 64) {
               float xt = 0.f;
@@ -583,6 +698,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bulk_commit();
           }
           ++nstore;
+          if (cs + 64 < kBN) tmem_ld_wait(n0, n1);
         }
         if (ce && row < g.M)
           g.stats[static_cast<int64_t>(nb) * g.stats_ld + row] =
@@ -594,7 +710,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int cs = 0; cs < kBN; cs += 32) {
           uint32_t v[32];
           tmem_ld32(t_row + cs, v);
-          tmem_ld_wait();
+          tmem_ld_wait(v);
           if (g.row_scale) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * rs);
@@ -625,7 +741,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int cc = 0; cc < kBN; cc += 32) {
           uint32_t v[32];
           tmem_ld32(t_row + cc, v);
-          tmem_ld_wait();
+          tmem_ld_wait(v);
           const int col0 = nb * kBN + cc;
           if (!row_ok || col0 >= g.n_limit) continue;
           const int ncols = min(32, g.n_limit - col0);  // a multiple of 8
