@@ -299,6 +299,34 @@ gh_status_t gh_profile_read(gh_kernel_t kind, double* total_ms, int64_t* launche
  * including the small counting/reduction kernels). */
 int64_t gh_launch_count(void);
 
+/*
+ * gh_debug_set — knobs for testing the library's failure path; the Greyhound
+ * API has no counterpart.  Every device-side wait in the library is bounded:
+ * when one runs out, the kernel records GH_ERR_TIMEOUT, all its roles stop,
+ * copies already in flight are waited for, TMEM is freed and the kernel
+ * returns.  These knobs make such a wait run out on purpose, so that path can
+ * be exercised without faulting or hanging the GPU:
+ *
+ *   GH_DEBUG_WAIT_LIMIT_NS       the wait limit of every later launch on the
+ *                                current device, in ns (value <= 0: back to the
+ *                                default of 2 s).  Synchronous.
+ *   GH_DEBUG_WITHHOLD_RING_PIECE the next launch of the two-pass cross-entropy
+ *                                ring leaves out the copy of piece `value` of
+ *                                its first CTA (-1: none); the launch resets it.
+ *   GH_DEBUG_WITHHOLD_GEMM_STAGE the next linear cross-entropy GEMM launch
+ *                                leaves out the operand loads of stage `value`
+ *                                of its first CTA (pair) (-1: none); the launch
+ *                                resets it.
+ * Off by default; not for production use.  Returns GH_ERR_INVALID_ARG for an
+ * unknown knob, GH_ERR_CUDA if the device copy fails.
+ */
+typedef enum {
+  GH_DEBUG_WAIT_LIMIT_NS = 0,
+  GH_DEBUG_WITHHOLD_RING_PIECE = 1,
+  GH_DEBUG_WITHHOLD_GEMM_STAGE = 2
+} gh_debug_t;
+gh_status_t gh_debug_set(gh_debug_t knob, int64_t value);
+
 /* Static, NUL-terminated description of a status code. */
 const char* gh_status_string(gh_status_t status);
 

@@ -101,6 +101,8 @@ def lib() -> ctypes.CDLL:
     L.gh_profile_read.restype = c_int
     L.gh_launch_count.argtypes = []
     L.gh_launch_count.restype = c_int64
+    L.gh_debug_set.argtypes = [c_int, c_int64]
+    L.gh_debug_set.restype = c_int
     _lib = L
     return L
 
@@ -465,6 +467,17 @@ def gh_profile_enable(enable: bool = True) -> None:
     _check(lib().gh_profile_enable(1 if enable else 0), "gh_profile_enable")
 
 
+GH_DEBUG = {"wait_limit_ns": 0, "withhold_ring_piece": 1, "withhold_gemm_stage": 2}
+
+
+def gh_debug_set(knob: str, value: int) -> None:
+    """Failure-path test knobs (off by default): the device wait limit in ns
+    (``wait_limit_ns``; <= 0 restores the default), or one copy the next ring
+    or GEMM launch leaves out (``withhold_ring_piece``, ``withhold_gemm_stage``;
+    -1 none)."""
+    _check(lib().gh_debug_set(GH_DEBUG[knob], int(value)), "gh_debug_set")
+
+
 def gh_profile_read(kind: str):
     """(summed milliseconds, launches) recorded for one kernel kind."""
     ms = ctypes.c_double(0.0)
@@ -488,7 +501,7 @@ __all__ = [
     "gh_ce_fwd_bwd", "gh_ce_fwd_bwd_noalloc", "GH_NOALLOC_MAX_ROWS", "gh_ce_fwd", "gh_selective_log_softmax",
     "gh_ce_vjp", "gh_linear_ce", "gh_chunked_linear_loss", "CHUNK_LOSS_FN",
     "gh_count_valid", "gh_ce_fwd_bwd_shard", "gh_linear_ce_shard",
-    "gh_get_device_status", "gh_profile_enable", "gh_profile_read",
+    "gh_get_device_status", "gh_profile_enable", "gh_profile_read", "gh_debug_set", "GH_DEBUG",
     "gh_launch_count", "GH_KERNEL",
     "GH_OK", "GH_ERR_INVALID_ARG", "GH_ERR_UNSUPPORTED", "GH_ERR_ALLOC", "GH_ERR_CUDA",
     "GH_ERR_TIMEOUT", "GH_ERR_TARGET_RANGE", "GH_REDUCTION", "GH_ACCUM", "GH_F32", "GH_BF16",

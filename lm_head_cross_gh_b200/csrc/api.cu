@@ -359,6 +359,23 @@ gh_status_t gh_profile_read(gh_kernel_t kind, double* total_ms, int64_t* launche
 
 int64_t gh_launch_count(void) { return launch_counter().load(); }
 
+gh_status_t gh_debug_set(gh_debug_t knob, int64_t value) {
+  switch (knob) {
+    case GH_DEBUG_WAIT_LIMIT_NS: {
+      const uint64_t v = value > 0 ? static_cast<uint64_t>(value) : kWaitTimeoutNs;
+      if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return GH_ERR_CUDA;
+      return GH_OK;
+    }
+    case GH_DEBUG_WITHHOLD_RING_PIECE:
+      debug_ring_piece().store(value >= 0 ? value : -1);
+      return GH_OK;
+    case GH_DEBUG_WITHHOLD_GEMM_STAGE:
+      debug_gemm_stage().store(value >= 0 && value < (int64_t(1) << 30) ? value : -1);
+      return GH_OK;
+  }
+  return GH_ERR_INVALID_ARG;
+}
+
 const char* gh_status_string(gh_status_t s) {
   switch (s) {
     case GH_OK: return "ok";

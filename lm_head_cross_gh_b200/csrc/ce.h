@@ -34,6 +34,7 @@ struct CeArgs {
   int congruent;                      // (logits - grad) % 16 == 0
   int profile_kind;                   // gh_kernel_t the row kernel is timed as
   int mode;                           // CeMode
+  int64_t withhold_plus1;             // failure-path tests: 1 + the piece CTA 0's ring producer leaves out (0: none)
 };
 
 struct CePlan {

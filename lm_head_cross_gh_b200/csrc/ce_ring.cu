@@ -513,6 +513,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
         for (int p = 0; p < np; ++p, ++n) {
           const int s = static_cast<int>(n % kRingSlots);
           if (!wait(&sh.empty[s], ((n / kRingSlots) & 1) ^ 1)) return false;
+          if (a.withhold_plus1 != 0 && blockIdx.x == 0 && n + 1 == a.withhold_plus1) continue;  // test of the failure path
           const int c0 = r.c_lo + p * kRingPieceChunks;
           const uint32_t bytes = 16u * static_cast<uint32_t>(tmin(kRingPieceChunks, r.c_hi - c0));
           mbar_arrive_expect_tx(&sh.full[s], bytes);
@@ -783,10 +784,12 @@ RingKernel ring_kernel_for(int es, int mode) {
 
 int ce_ring_smem_bytes() { return kRingHdrBytes + kRingSlots * kRingPieceBytes; }
 
-gh_status_t ce_ring_launch(const CeArgs& a, int es, int grid, cudaStream_t stream) {
+gh_status_t ce_ring_launch(const CeArgs& args, int es, int grid, cudaStream_t stream) {
+  CeArgs a = args;
   const bool long_rows = a.V * es >= kLongRowBytes;
   RingKernel kern;
   if (a.mode == kModeFwdBwd) {
+    a.withhold_plus1 = debug_ring_piece().exchange(-1) + 1;
     if (es == 4) kern = long_rows ? ce_ring2_kernel<float, true> : ce_ring2_kernel<float, false>;
     else kern = long_rows ? ce_ring2_kernel<uint16_t, true> : ce_ring2_kernel<uint16_t, false>;
   } else {

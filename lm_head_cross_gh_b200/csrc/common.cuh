@@ -24,9 +24,15 @@ __device__ __forceinline__ void record_status(int code) {
   atomicCAS(&g_device_status, 0, code);
 }
 
-// Every device-side wait gives up after kWaitTimeoutNs of wall time (read
-// from %globaltimer): far above any legitimate wait, yet finite.
+// Every device-side wait gives up after wait_limit_ns() of wall time (read
+// from %globaltimer): by default kWaitTimeoutNs, far above any legitimate wait,
+// yet finite.  gh_debug_set can lower it (tests of the failure path).
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
+__device__ uint64_t g_wait_limit_ns = kWaitTimeoutNs;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+  return *reinterpret_cast<const volatile uint64_t*>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
@@ -85,14 +91,14 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for phase `parity` of `bar` to complete.  Returns false (and
-// records GH_ERR_TIMEOUT) once kWaitTimeoutNs has passed.
+// records GH_ERR_TIMEOUT) once wait_limit_ns() has passed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity, 100000u)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(a, parity, 100000u)) return true;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) break;
+    if (global_timer_ns() - t0 > wait_limit_ns()) break;
   }
   record_status(GH_ERR_TIMEOUT);
   return false;
@@ -214,7 +220,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (try_once()) return true;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) break;
+    if (global_timer_ns() - t0 > wait_limit_ns()) break;
   }
   record_status(GH_ERR_TIMEOUT);
   return false;

@@ -63,6 +63,7 @@ struct GemmCfg {
   static constexpr int kSmem = 1024 /*align*/ + kStages * kStageBytes + kOutBytes + 256 /*barriers*/;
 };
 constexpr int kGemmSmem = GemmCfg<false>::kSmem;
+constexpr int kMaxSplits = 4;  // K splits a tile may be cut into when they are summed in the kernel
 static_assert(GemmCfg<true>::kSmem <= 232448 && GemmCfg<false>::kSmem <= 232448, "shared memory per CTA");
 
 // Epilogue modes (what happens to the fp32 tile).  The first three go out
@@ -73,8 +74,9 @@ enum GemmEpi : int {
   kEpiStoreF32 = 1,   // out(f32)  = tile                       TMA store
   kEpiAddF32 = 2,     // out(f32) += tile                       TMA reduce-add (in L2)
   kEpiBf16Add = 3,    // out = bf16(float(out) + tile), direct loads and stores (bf16 accumulator)
-  kEpiCeExp = 4       // logits tile of the fused cross-entropy: out(bf16) = exp(tile - R_row)
+  kEpiCeExp = 4,      // logits tile of the fused cross-entropy: out(bf16) = exp(tile - R_row)
                       // (0 for ignored rows), plus per (row, column tile) sum and max
+  kEpiAccToBf16 = 5   // out(bf16) = bf16(acc + tile), acc an fp32 [M, acc_ld] array   TMA store
 };
 
 struct GemmArgs {
@@ -99,6 +101,21 @@ struct GemmArgs {
   float* x_target;         // [M]: the fp32 logit at the row's target column (valid rows)
   const float* row_ref;    // [M] R_row, or null for R_row = 0
   const int* run_flag;     // non-null: the kernel does nothing unless *run_flag != 0
+  // kEpiStoreF32 with k_splits > 1 and split_out non-null: the K splits are
+  // summed in the kernel.  Each split stores its fp32 partial (rows
+  // ks * split_rows + r of split_ws, row stride N); the last split to finish a
+  // 32-row slice of a tile adds the slice's partials in split order (the same
+  // order whichever split finishes last) and writes bf16 rows of split_out.
+  const float* split_ws;
+  uint16_t* split_out;
+  int64_t split_ld;
+  int* split_count;        // one counter per (tile, CTA of the pair, 32-row slice), 0 between launches
+  // kEpiAccToBf16
+  const float* acc;
+  int64_t acc_ld;
+  // failure-path tests: 1 + the stage of unit 0's first tile whose loads the
+  // producer leaves out (0: none)
+  int withhold_plus1;
 };
 
 // ---- PTX wrappers ----------------------------------------------------------------
@@ -286,7 +303,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   while (true) {
     if (test()) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > wait_limit_ns()) {
       *abort_flag = 1;
       record_status(GH_ERR_TIMEOUT);
       return false;
@@ -307,6 +324,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                      const __grid_constant__ CUtensorMap tma_out, GemmArgs g) {
   using C = GemmCfg<PAIR>;
+  // Each operand layout serves one contraction, so each instantiation keeps
+  // only the epilogues that contraction uses (fewer live registers).
+  constexpr bool kLogits = !A_MN && !B_MN;  // kEpiCeExp, kEpiStoreBf16
+  constexpr bool kDx = !A_MN && B_MN;       // kEpiStoreBf16 (row scale), kEpiStoreF32 (+ split sums)
+  constexpr bool kDw = A_MN && B_MN;        // kEpiStoreBf16, kEpiStoreF32, kEpiAddF32, kEpiBf16Add, kEpiAccToBf16
   constexpr int kStages = C::kStages;
   constexpr int kStageBytes = C::kStageBytes;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -404,6 +426,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = stage_base + stage * kStageBytes;
           uint8_t* sb = sa + kABytes;
           const int k0 = kb * kBK;
+          if (g.withhold_plus1 != 0 && unit == 0 && leader && issued + 1 == static_cast<uint32_t>(g.withhold_plus1)) {
+            // test of the failure path: this stage's barrier is never armed,
+            // so the MMA issuer's bounded wait for it runs out
+            ++issued;
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
+          }
           auto load = [&](void* dst, const CUtensorMap* map, int x, int y) {
             if constexpr (PAIR) {
               if (!leader) {
@@ -442,7 +474,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t t0 = global_timer_ns();
           for (uint32_t n = (issued > kStages ? issued - kStages : 0); n < issued; ++n) {
             const uint32_t a = smem_u32(&full[n % kStages]);
-            while (!mbar_try_wait(a, (n / kStages) & 1, 20000u) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+            while (!mbar_try_wait(a, (n / kStages) & 1, 20000u) && global_timer_ns() - t0 < wait_limit_ns()) {
             }
           }
         }
@@ -536,7 +568,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         ++nstore;
       };
-      if (g.epi == kEpiCeExp && g.N - nb * kBN >= kBN) {
+      if (kLogits && g.epi == kEpiCeExp && g.N - nb * kBN >= kBN) {
         // A whole tile of the fused cross-entropy: every column is inside N.
         // exp(x - R) = 2^(x log2 e - R log2 e) with packed f32x2 arithmetic; a
         // reference of -inf stores 0 for rows that are ignored or past M.
@@ -602,10 +634,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (row < g.M)
           g.stats[static_cast<int64_t>(nb) * g.stats_ld + row] =
               make_float2((sA.x + sA.y) + (sB.x + sB.y), fmaxf(mA, mB));
-      } else if (g.epi == kEpiStoreBf16 || g.epi == kEpiCeExp) {
+      } else if (g.epi == kEpiStoreBf16 || (kLogits && g.epi == kEpiCeExp)) {
         // The bf16 store (optionally row-scaled), and the fused cross-entropy's
         // last column tile, whose columns past N are left out of the sum and max.
-        const bool ce = g.epi == kEpiCeExp;
+        const bool ce = kLogits && g.epi == kEpiCeExp;
         float rs = 1.0f, nrl2 = 0.0f;
         int tcol = -1;       // target column relative to the tile (-1: none)
         bool keep = true;    // row stores its exponentials (valid row)
@@ -703,7 +735,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (ce && row < g.M)
           g.stats[static_cast<int64_t>(nb) * g.stats_ld + row] =
               make_float2((s0 + s1) + (s2 + s3), fmaxf(m0, m1));
-      } else if (g.epi == kEpiStoreF32 || g.epi == kEpiAddF32) {
+      } else if (kDw && g.epi == kEpiAccToBf16) {
+        // the fp32 accumulator's rows plus this tile, rounded once to bf16
+#pragma unroll 1
+        for (int cs = 0; cs < kBN; cs += 64) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(t_row + cs, v0);
+          tmem_ld32(t_row + cs + 32, v1);
+          tmem_ld_wait(v0, v1);
+          const int col = nb * kBN + cs;
+          if (row < g.M) {
+            const float* a = g.acc + static_cast<int64_t>(row) * g.acc_ld + col;
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) {
+              if (col + j < g.N) {  // N is a multiple of 8
+                const float4 p = __ldcs(reinterpret_cast<const float4*>(a + j));
+                uint32_t* w = j < 32 ? &v0[j] : &v1[j - 32];
+                w[0] = __float_as_uint(__uint_as_float(w[0]) + p.x);
+                w[1] = __float_as_uint(__uint_as_float(w[1]) + p.y);
+                w[2] = __float_as_uint(__uint_as_float(w[2]) + p.z);
+                w[3] = __float_as_uint(__uint_as_float(w[3]) + p.w);
+              }
+            }
+          }
+          uint32_t pk[32];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            pk[j / 2] = pack_bf16x2(__uint_as_float(v0[j]), __uint_as_float(v0[j + 1]));
+            pk[16 + j / 2] = pack_bf16x2(__uint_as_float(v1[j]), __uint_as_float(v1[j + 1]));
+          }
+          store_slice(pk, col);
+        }
+      } else if (!kLogits && (g.epi == kEpiStoreF32 || g.epi == kEpiAddF32)) {
         // 32-column slices: 1 TMEM load -> 32 rows x 128 bytes of fp32
         const float rs = g.row_scale ? (row < g.M ? g.row_scale[row] : 0.0f) : 1.0f;
 #pragma unroll 1
@@ -734,7 +797,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           ++nstore;
         }
-      } else {
+      } else if (kDw) {
         // kEpiBf16Add: accumulate into the bf16 output with plain loads and stores
         const bool row_ok = row < g.m_limit;
 #pragma unroll 1
@@ -769,6 +832,59 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) {
         if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(&tmem_empty[acc], 0));
         else mbar_arrive(&tmem_empty[acc]);
+      }
+      if (kDx && g.epi == kEpiStoreF32 && g.k_splits > 1 && g.split_out) {
+        // this warp's partial rows are written (not only read out of shared
+        // memory) before the slice's count goes up
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
+        const int cidx = ((mb * g.tiles_n + nb) * (PAIR ? 2 : 1) + static_cast<int>(rank)) * 4 + q;
+        int last = 0;
+        if (lane == 0) {
+          __threadfence();
+          last = atomicAdd(&g.split_count[cidx], 1) == g.k_splits - 1;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();  // every split's partial of this slice is visible
+          if (lane == 0) g.split_count[cidx] = 0;
+          const int col = nb * kBN + 8 * lane;  // lanes across the row: coalesced 32-byte reads
+          if (col < g.N) {
+            // 2 rows at a time with every split's loads issued before the adds
+#pragma unroll 1
+            for (int r0 = 0; r0 < 32; r0 += 2) {
+              float4 u[kMaxSplits][2][2];
+#pragma unroll
+              for (int sp = 0; sp < kMaxSplits; ++sp) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                  const int rr = rbase + r0 + i;
+                  if (sp < g.k_splits && rr < g.M) {
+                    const float* p = g.split_ws + (static_cast<int64_t>(sp) * g.split_rows + rr) * g.N + col;
+                    u[sp][i][0] = __ldcg(reinterpret_cast<const float4*>(p));
+                    u[sp][i][1] = __ldcg(reinterpret_cast<const float4*>(p + 4));
+                  }
+                }
+              }
+#pragma unroll
+              for (int i = 0; i < 2; ++i) {
+                const int rr = rbase + r0 + i;
+                if (rr >= g.M) break;
+                float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int sp = 0; sp < kMaxSplits; ++sp) {
+                  if (sp < g.k_splits) {
+                    a[0] += u[sp][i][0].x; a[1] += u[sp][i][0].y; a[2] += u[sp][i][0].z; a[3] += u[sp][i][0].w;
+                    a[4] += u[sp][i][1].x; a[5] += u[sp][i][1].y; a[6] += u[sp][i][1].z; a[7] += u[sp][i][1].w;
+                  }
+                }
+                *reinterpret_cast<uint4*>(g.split_out + static_cast<int64_t>(rr) * g.split_ld + col) =
+                    make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                               pack_bf16x2(a[6], a[7]));
+              }
+            }
+          }
+        }
       }
       if (++acc == 2) {
         acc = 0;

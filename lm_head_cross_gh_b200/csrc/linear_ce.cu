@@ -21,11 +21,13 @@
 //                                     row factor applied in its epilogue
 //   5  dW    (+)= P^T Xs_c            tcgen05 GEMM (both operands M/N-major);
 //                                     fp32 accumulator across chunks (TMA store,
-//                                     then TMA reduce-add in L2), rounded once to
-//                                     bf16 at the end ("fp32"), or accumulated in
-//                                     the bf16 output ("weight")
-// When the dX tiles alone would leave SMs idle, dX splits K into fp32 partials
-// that a second kernel sums in a fixed order (deterministic).
+//                                     then TMA reduce-add in L2; the last chunk
+//                                     adds it and rounds once to bf16, "fp32"),
+//                                     or accumulated in the bf16 output ("weight")
+// When the dX tiles alone would leave SMs idle, dX splits K into fp32 partials;
+// inside the same kernel the last split to finish each 32-row slice sums them in
+// split order (deterministic) and writes the bf16 rows.  With fp32 accumulation
+// the last chunk's dW epilogue adds the accumulator and rounds once to bf16.
 //
 // gh_chunked_linear_loss (a caller-provided loss per chunk) keeps the plain
 // form: step 1 stores the bf16 logits, the caller's callback overwrites them
@@ -87,36 +89,7 @@ bool make_out_f32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows
   return make_tmap(m, base, cols, rows, ld * 4, 32, true, 32);
 }
 
-// out[r, c] = bf16(sum_s ws[s][r, c]) for r < rows, in split order (deterministic).
-__global__ void splitk_reduce_kernel(const float* __restrict__ ws, int splits, int64_t split_stride, int rows,
-                                     int cols, uint16_t* __restrict__ out, int64_t ld_out) {
-  pdl_wait();
-  pdl_trigger();
-  const int64_t n4 = static_cast<int64_t>(rows) * (cols / 4);
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / (cols / 4), c4 = i - r * (cols / 4);
-    float4 a = *reinterpret_cast<const float4*>(ws + r * cols + 4 * c4);
-    for (int sp = 1; sp < splits; ++sp) {
-      const float4 b = *reinterpret_cast<const float4*>(ws + sp * split_stride + r * cols + 4 * c4);
-      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-    }
-    *reinterpret_cast<uint2*>(out + r * ld_out + 4 * c4) = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
-  }
-}
-
-// out = bf16(acc), the fp32 weight-gradient accumulator's single final rounding.
-__global__ void cast_bf16_kernel(const float* __restrict__ acc, int64_t n4, uint16_t* __restrict__ out) {
-  pdl_wait();
-  pdl_trigger();
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[i];
-    reinterpret_cast<uint2*>(out)[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
-  }
-}
-
-// Per-chunk step 2 of the fused cross-entropy (one CTA of 256 threads per 32
+// Per-chunk step 2 of the fused cross-entropy (one CTA of 512 threads per 32
 // rows).  Each row's statistics are combined over the column tiles in a fixed
 // order (deterministic): S = sum of the tiles' sums of exp(x - R), M = max.
 struct FinalizeArgs {
@@ -148,9 +121,11 @@ constexpr float kLseWindow = 40.0f;
 // of the target entry alone is scale * 2^-9).
 constexpr float kZFactorFloor = 9.5367431640625e-07f;  // 2^-20
 
-__global__ void __launch_bounds__(256) lce_finalize_kernel(FinalizeArgs a) {
-  __shared__ float sh_s[8][32];
-  __shared__ float sh_m[8][32];
+constexpr int kFinWarps = 16;
+
+__global__ void __launch_bounds__(kFinWarps * 32) lce_finalize_kernel(FinalizeArgs a) {
+  __shared__ float sh_s[kFinWarps][32];
+  __shared__ float sh_m[kFinWarps][32];
   __shared__ float sh_alpha[32];
   pdl_wait();
   pdl_trigger();
@@ -160,7 +135,8 @@ __global__ void __launch_bounds__(256) lce_finalize_kernel(FinalizeArgs a) {
   const int row = row0 + lane;
   float s = 0.0f, m = -INFINITY;
   if (row < a.rows) {
-    for (int nb = warp; nb < a.tiles_n; nb += 8) {
+#pragma unroll 4
+    for (int nb = warp; nb < a.tiles_n; nb += kFinWarps) {
       const float2 v = a.stats[static_cast<int64_t>(nb) * a.stats_ld + row];
       s += v.x;
       m = fmaxf(m, v.y);
@@ -174,7 +150,7 @@ __global__ void __launch_bounds__(256) lce_finalize_kernel(FinalizeArgs a) {
     if (row < a.rows) {
       float S = 0.0f, M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
+      for (int w = 0; w < kFinWarps; ++w) {
         S += sh_s[w][lane];
         M = fmaxf(M, sh_m[w][lane]);
       }
@@ -209,7 +185,7 @@ __global__ void __launch_bounds__(256) lce_finalize_kernel(FinalizeArgs a) {
   // Xs = bf16(alpha X) for this block's rows, 16-byte vectors
   const int d8 = a.D / 8;
   const int nrows = min(32, a.rows - row0);
-  for (int i = threadIdx.x; i < nrows * d8; i += 256) {
+  for (int i = threadIdx.x; i < nrows * d8; i += kFinWarps * 32) {
     const int r = i / d8, c = i - r * d8;
     const int64_t off = static_cast<int64_t>(row0 + r) * a.D + 8 * c;
     const uint4 x = *reinterpret_cast<const uint4*>(a.X + off);
@@ -240,6 +216,8 @@ gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
                         const sm100::GemmArgs& g, bool pair, int kind, cudaStream_t stream) {
   const int tiles = g.tiles_m * g.tiles_n * g.k_splits;
   if (tiles == 0) return GH_OK;
+  sm100::GemmArgs ga = g;
+  if (!g.run_flag) ga.withhold_plus1 = static_cast<int>(debug_gemm_stage().exchange(-1) + 1);
   cudaError_t e;
   if (pair) {
     auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN, true>;
@@ -247,14 +225,14 @@ gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
     const int pairs = std::min(tiles, std::max(1, sm_count() / 2));
     ProfileScope prof(kind, stream);
     e = launch_pdl(kern, dim3(2 * pairs), dim3(sm100::kGemmThreads), sm100::GemmCfg<true>::kSmem, stream, 2, ta, tb,
-                   tout, g);
+                   tout, ga);
   } else {
     auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN, false>;
     if (ensure_smem_limit(kern, sm100::GemmCfg<false>::kSmem) != cudaSuccess) return GH_ERR_CUDA;
     const int grid = std::min(tiles, sm_count());
     ProfileScope prof(kind, stream);
     e = launch_pdl(kern, dim3(grid), dim3(sm100::kGemmThreads), sm100::GemmCfg<false>::kSmem, stream, 1, ta, tb,
-                   tout, g);
+                   tout, ga);
   }
   note_launch();
   return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
@@ -329,7 +307,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const int tiles_m_max = static_cast<int>((chunk + tile_m - 1) / tile_m);
   const int dx_num_kb = static_cast<int>((V + sm100::kBK - 1) / sm100::kBK);
   const int dx_tiles_max = tiles_m_max * static_cast<int>((D + sm100::kBN - 1) / sm100::kBN);
-  const int dx_splits = choose_splits(dx_tiles_max, dx_num_kb, units);
+  const int dx_splits = std::min(sm100::kMaxSplits, choose_splits(dx_tiles_max, dx_num_kb, units));
   const int64_t rows_pad = static_cast<int64_t>(tiles_m_max) * tile_m;
 
   const bool custom = a.loss_fn != nullptr;
@@ -356,7 +334,10 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const size_t xs_bytes = fused ? static_cast<size_t>(rows_pad) * D * 2 : 0;
   const size_t off_flags = up(off_xs + xs_bytes);
   const size_t flags_bytes = fused ? static_cast<size_t>(nchunks) * sizeof(int) : 0;
-  const size_t total = off_flags + flags_bytes;
+  const size_t off_count = up(off_flags + flags_bytes);
+  const size_t count_bytes =
+      dx_splits > 1 ? static_cast<size_t>(dx_tiles_max) * 2 /*CTAs of a pair*/ * 4 /*slices*/ * sizeof(int) : 0;
+  const size_t total = off_count + count_bytes;
   void* scratch = nullptr;
   gh_status_t st = scratch_alloc(&scratch, total, stream);
   if (st != GH_OK) return st;
@@ -373,6 +354,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   float* alpha = fused ? reinterpret_cast<float*>(base + off_alpha) : nullptr;
   uint16_t* Xs = fused ? reinterpret_cast<uint16_t*>(base + off_xs) : nullptr;
   int* flags = fused ? reinterpret_cast<int*>(base + off_flags) : nullptr;
+  int* split_count = dx_splits > 1 ? reinterpret_cast<int*>(base + off_count) : nullptr;
 
   const uint16_t* X = static_cast<const uint16_t*>(a.X);
   const uint16_t* W = static_cast<const uint16_t*>(a.W);
@@ -383,6 +365,8 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
        : a.n_total ? GH_OK
                    : ce_count_launch(a.targets, N, V, a.ignore_index, counter, stream);
   if (st == GH_OK && fused && cudaMemsetAsync(flags, 0, flags_bytes, stream) != cudaSuccess) st = GH_ERR_CUDA;
+  if (st == GH_OK && split_count && cudaMemsetAsync(split_count, 0, count_bytes, stream) != cudaSuccess)
+    st = GH_ERR_CUDA;
   // W as the K-major B operand of the logits GEMM and the N-major B operand of
   // dX; the weight-gradient output (bf16) and accumulator (fp32) maps.
   CUtensorMap tm_w_k, tm_w_n, tm_dw_out, tm_acc, tm_ws;
@@ -442,7 +426,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       const dim3 fgrid(static_cast<unsigned>((rows + 31) / 32));
       {
         ProfileScope prof(GH_KERNEL_CHUNK_CE, stream);
-        const cudaError_t e = launch_pdl(lce_finalize_kernel, fgrid, dim3(256), 0, stream, 1, fa);
+        const cudaError_t e = launch_pdl(lce_finalize_kernel, fgrid, dim3(kFinWarps * 32), 0, stream, 1, fa);
         note_launch();
         if (e != cudaSuccess) {
           st = GH_ERR_CUDA;
@@ -458,7 +442,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       fa.recompute = 1;
       {
         ProfileScope prof(GH_KERNEL_CHUNK_CE, stream);
-        const cudaError_t e = launch_pdl(lce_finalize_kernel, fgrid, dim3(256), 0, stream, 1, fa);
+        const cudaError_t e = launch_pdl(lce_finalize_kernel, fgrid, dim3(kFinWarps * 32), 0, stream, 1, fa);
         note_launch();
         if (e != cudaSuccess) {
           st = GH_ERR_CUDA;
@@ -485,16 +469,13 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       g3.k_splits = (g3.num_kb + g3.kb_per_split - 1) / g3.kb_per_split;
       g3.split_rows = static_cast<int>(rows_pad);
       g3.epi = sm100::kEpiStoreF32;
+      // the last split to finish each 32-row slice sums the partials in split order
+      g3.split_ws = ws;
+      g3.split_out = dX + c0 * D;
+      g3.split_ld = D;
+      g3.split_count = split_count;
       st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_ws, g3, pair, GH_KERNEL_DX_GEMM, stream);
       if (st != GH_OK) break;
-      const cudaError_t e = launch_pdl(splitk_reduce_kernel, dim3(sms * 4), dim3(256), 0, stream, 1,
-                                       static_cast<const float*>(ws), g3.k_splits, rows_pad * D, rows,
-                                       static_cast<int>(D), dX + c0 * D, D);
-      note_launch();
-      if (e != cudaSuccess) {
-        st = GH_ERR_CUDA;
-        break;
-      }
     } else {
       st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_dx_out, g3, pair, GH_KERNEL_DX_GEMM, stream);
       if (st != GH_OK) break;
@@ -506,22 +487,20 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     g4.ld_out = D;
     const CUtensorMap* out4 = &tm_dw_out;
     if (a.accum == GH_ACCUM_FP32) {
-      if (acc32) {
+      if (acc32 && c + 1 < nchunks) {
         g4.epi = c == 0 ? sm100::kEpiStoreF32 : sm100::kEpiAddF32;
         out4 = &tm_acc;
+      } else if (acc32) {
+        // the last chunk adds its product to the fp32 accumulator and rounds
+        // the sum to bf16 once, straight into grad_weight
+        g4.epi = sm100::kEpiAccToBf16;
+        g4.acc = acc;
+        g4.acc_ld = D;
       }
     } else {
       g4.epi = c == 0 ? sm100::kEpiStoreBf16 : sm100::kEpiBf16Add;
     }
     st = launch_gemm<true, true>(tm_l_m, tm_x_n, *out4, g4, pair, GH_KERNEL_DW_GEMM, stream);
-  }
-  if (st == GH_OK && acc32) {
-    // the fp32 accumulator's single rounding to the weight dtype
-    const int64_t n4 = V * D / 4;
-    const cudaError_t e =
-        launch_pdl(cast_bf16_kernel, dim3(sms * 4), dim3(256), 0, stream, 1, static_cast<const float*>(acc), n4, dW);
-    note_launch();
-    if (e != cudaSuccess) st = GH_ERR_CUDA;
   }
   if (st == GH_OK && !custom) st = ce_reduce_launch(row_loss, N, n_valid, a.mean, a.loss, stream);
   scratch_free(scratch, stream);

@@ -50,6 +50,19 @@ inline std::atomic<long long>& launch_counter() {
 
 inline void note_launch(int n = 1) { launch_counter().fetch_add(n, std::memory_order_relaxed); }
 
+// Failure-path test knobs (gh_debug_set): each names one copy that the next
+// launch of its kernel leaves out, so that a consumer's bounded wait runs
+// out.  -1 (the default) leaves nothing out; a launch takes the value and
+// resets it.
+inline std::atomic<long long>& debug_ring_piece() {
+  static std::atomic<long long> v{-1};
+  return v;
+}
+inline std::atomic<long long>& debug_gemm_stage() {
+  static std::atomic<long long> v{-1};
+  return v;
+}
+
 class ProfileScope {
  public:
   ProfileScope(int kind, cudaStream_t stream) : stream_(stream) {
