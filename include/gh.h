@@ -158,6 +158,26 @@ gh_status_t gh_linear_ce_shard(const void* inputs, const void* weight, const int
                                void* grad_inputs, void* grad_weight, void* stream);
 
 /*
+ * gh_linear_ce_shard_f32 — gh_linear_ce_shard with fp32 accumulation
+ * (Greyhound `grad_weight_accum_dtype` "fp32": accumulate in fp32, cast once)
+ * whose weight gradient is returned unrounded, so that a data-parallel caller
+ * can sum the shards' fp32 accumulators (all-reduce in fp32) and round the
+ * batch's sum once, with gh_cast_f32_to_bf16.
+ *   grad_weight_f32  [V, D] float32, device, 16-byte aligned, written (not
+ *                    added to) with this shard's sum over its chunks of
+ *                    G_c^T @ inputs[chunk], in fp32.
+ * Other arguments as for gh_linear_ce_shard (no accum_dtype argument).
+ *
+ * gh_cast_f32_to_bf16 — dst[i] = bf16(src[i]) (round to nearest even) for
+ * n elements; src 16-byte aligned, dst 8-byte aligned, device.
+ */
+gh_status_t gh_linear_ce_shard_f32(const void* inputs, const void* weight, const int64_t* targets, int64_t N,
+                                   int64_t D, int64_t V, int64_t chunk, int64_t ignore_index,
+                                   gh_reduction_t reduction, float z_mult, const int64_t* n_valid_total,
+                                   float* loss, void* grad_inputs, float* grad_weight_f32, void* stream);
+gh_status_t gh_cast_f32_to_bf16(const float* src, void* dst, int64_t n, void* stream);
+
+/*
  * gh_ce_fwd — the cross-entropy loss of gh_ce_fwd_bwd without its gradient:
  * the evaluation form (forward only, nothing kept for a backward), reading the
  * logits once.

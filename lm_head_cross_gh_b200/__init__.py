@@ -75,6 +75,11 @@ def lib() -> ctypes.CDLL:
     L.gh_linear_ce_shard.argtypes = [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64, c_int,
                                      c_int64, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
     L.gh_linear_ce_shard.restype = c_int
+    L.gh_linear_ce_shard_f32.argtypes = [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64,
+                                         c_int64, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
+    L.gh_linear_ce_shard_f32.restype = c_int
+    L.gh_cast_f32_to_bf16.argtypes = [c_void_p, c_void_p, c_int64, c_void_p]
+    L.gh_cast_f32_to_bf16.restype = c_int
     L.gh_ce_fwd.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_int, c_float,
                             c_void_p, c_void_p, c_void_p]
     L.gh_ce_fwd.restype = c_int
@@ -274,6 +279,51 @@ def gh_linear_ce_shard(inputs, weight, targets, n_valid_total, ignore_index: int
                                   _ptr(loss), _ptr(grad_inputs), _ptr(grad_weight), _stream_handle(stream))
     _check(st, "gh_linear_ce_shard")
     return loss, grad_inputs, grad_weight
+
+
+def gh_linear_ce_shard_f32(inputs, weight, targets, n_valid_total, ignore_index: int = -100,
+                           reduction: str = "mean", z_loss: float = 0.0, chunk: int = 0, *, grad_inputs=None,
+                           grad_weight_f32=None, loss=None, stream=None):
+    """``gh_linear_ce_shard`` with fp32 accumulation whose weight gradient comes
+    back as the shard's unrounded fp32 sum (float32 [V, D]), for an fp32
+    cross-rank sum followed by one rounding (``gh_cast_f32_to_bf16``)."""
+    import torch
+    _need(inputs.dim() == 2 and weight.dim() == 2 and inputs.shape[1] == weight.shape[1], "shapes")
+    _need(inputs.dtype == torch.bfloat16 and weight.dtype == torch.bfloat16, "inputs/weight must be bfloat16")
+    _need(inputs.is_cuda and weight.is_cuda and inputs.is_contiguous() and weight.is_contiguous(), "layout")
+    _need(targets.dtype == torch.int64 and targets.is_cuda and targets.is_contiguous()
+          and targets.shape == (inputs.shape[0],), "targets: contiguous CUDA int64 [N]")
+    _need(n_valid_total.dtype == torch.int64 and n_valid_total.numel() == 1 and n_valid_total.is_cuda,
+          "n_valid_total: CUDA int64 scalar")
+    _need(reduction in GH_REDUCTION, "reduction")
+    N, D = inputs.shape
+    V = weight.shape[0]
+    if grad_inputs is None:
+        grad_inputs = torch.empty_like(inputs)
+    if grad_weight_f32 is None:
+        grad_weight_f32 = torch.empty((V, D), dtype=torch.float32, device=weight.device)
+    _need(grad_weight_f32.dtype == torch.float32 and grad_weight_f32.shape == (V, D)
+          and grad_weight_f32.is_contiguous(), "grad_weight_f32: contiguous float32 [V, D]")
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=inputs.device)
+    st = lib().gh_linear_ce_shard_f32(_ptr(inputs), _ptr(weight), _ptr(targets), N, D, V, int(chunk),
+                                      int(ignore_index), GH_REDUCTION[reduction], float(z_loss),
+                                      _ptr(n_valid_total), _ptr(loss), _ptr(grad_inputs), _ptr(grad_weight_f32),
+                                      _stream_handle(stream))
+    _check(st, "gh_linear_ce_shard_f32")
+    return loss, grad_inputs, grad_weight_f32
+
+
+def gh_cast_f32_to_bf16(src, out=None, stream=None):
+    """bf16 copy of a float32 CUDA tensor, rounded to nearest even by the library."""
+    import torch
+    _need(src.dtype == torch.float32 and src.is_cuda and src.is_contiguous(), "src: contiguous CUDA float32")
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    _need(out.dtype == torch.bfloat16 and out.numel() == src.numel() and out.is_contiguous(), "out")
+    _check(lib().gh_cast_f32_to_bf16(_ptr(src), _ptr(out), src.numel(), _stream_handle(stream)),
+           "gh_cast_f32_to_bf16")
+    return out
 
 
 def gh_ce_fwd(logits, targets, ignore_index: int = -100, reduction: str = "mean", z_loss: float = 0.0, *,
@@ -500,7 +550,8 @@ __all__ = [
     "GhError", "lib", "header_symbols", "status_string", "gh_status_string", "gh_version",
     "gh_ce_fwd_bwd", "gh_ce_fwd_bwd_noalloc", "GH_NOALLOC_MAX_ROWS", "gh_ce_fwd", "gh_selective_log_softmax",
     "gh_ce_vjp", "gh_linear_ce", "gh_chunked_linear_loss", "CHUNK_LOSS_FN",
-    "gh_count_valid", "gh_ce_fwd_bwd_shard", "gh_linear_ce_shard",
+    "gh_count_valid", "gh_ce_fwd_bwd_shard", "gh_linear_ce_shard", "gh_linear_ce_shard_f32",
+    "gh_cast_f32_to_bf16",
     "gh_get_device_status", "gh_profile_enable", "gh_profile_read", "gh_debug_set", "GH_DEBUG",
     "gh_launch_count", "GH_KERNEL",
     "GH_OK", "GH_ERR_INVALID_ARG", "GH_ERR_UNSUPPORTED", "GH_ERR_ALLOC", "GH_ERR_CUDA",

@@ -116,6 +116,12 @@ struct GemmArgs {
   // failure-path tests: 1 + the stage of unit 0's first tile whose loads the
   // producer leaves out (0: none)
   int withhold_plus1;
+  // Start without waiting for the previous kernel on the stream, and wait for
+  // it before exiting: for a GEMM that reads nothing the previous kernel
+  // writes, when that kernel waited for everything this one reads before it
+  // let dependents launch (so this GEMM fills SMs as the previous one's CTAs
+  // retire, and still completes after it).
+  int defer_wait;
 };
 
 // ---- PTX wrappers ----------------------------------------------------------------
@@ -379,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
-  pdl_wait();     // operands and outputs are free of the predecessor kernel from here on
+  if (!g.defer_wait) pdl_wait();  // operands and outputs are free of the predecessor kernel from here on
   pdl_trigger();  // one CTA per SM, all resident: the next kernel may start its prologue
   // A conditional launch whose flag is clear has no tile to compute (the flag
   // was written by a kernel that completed before pdl_wait returned).
@@ -896,6 +902,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   // ---------------- teardown ----------------
   __syncwarp();
+  if (g.defer_wait) pdl_wait();  // complete only after the previous kernel
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) {  // neither CTA leaves while the other may still signal it or read its tiles

@@ -196,6 +196,19 @@ __global__ void __launch_bounds__(kFinWarps * 32) lce_finalize_kernel(FinalizeAr
   }
 }
 
+__global__ void cast_f32_bf16_kernel(const float* __restrict__ src, int64_t n, uint16_t* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t n4 = n / 4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
+    const float4 v = reinterpret_cast<const float4*>(src)[i];
+    reinterpret_cast<uint2*>(out)[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+  for (int64_t i = 4 * n4 + blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n; i += stride)
+    out[i] = to_bf16_bits(src[i]);
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -286,12 +299,25 @@ int64_t default_chunk(int64_t N, int64_t ld) {
 
 }  // namespace
 
+gh_status_t cast_f32_bf16_launch(const float* src, void* out, int64_t n, cudaStream_t stream) {
+  if (n == 0) return GH_OK;
+  const int64_t blocks = std::min<int64_t>((n / 4 + 255) / 256 + 1, static_cast<int64_t>(sm_count()) * 8);
+  const cudaError_t e = launch_pdl(cast_f32_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, 1,
+                                   src, n, static_cast<uint16_t*>(out));
+  note_launch();
+  return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+}
+
 gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const int64_t N = a.N, D = a.D, V = a.V;
   if (N == 0) {
     // No token: zero loss, zero weight gradient.
     if (cudaMemsetAsync(a.loss, 0, sizeof(float), stream) != cudaSuccess) return GH_ERR_CUDA;
-    if (cudaMemsetAsync(a.dW, 0, static_cast<size_t>(V) * D * 2, stream) != cudaSuccess) return GH_ERR_CUDA;
+    if (a.dW32) {
+      if (cudaMemsetAsync(a.dW32, 0, static_cast<size_t>(V) * D * 4, stream) != cudaSuccess) return GH_ERR_CUDA;
+    } else if (cudaMemsetAsync(a.dW, 0, static_cast<size_t>(V) * D * 2, stream) != cudaSuccess) {
+      return GH_ERR_CUDA;
+    }
     return GH_OK;
   }
   if (!tensor_map_encoder()) return GH_ERR_UNSUPPORTED;
@@ -299,7 +325,10 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   int64_t chunk = a.chunk > 0 ? std::min<int64_t>(a.chunk, N) : default_chunk(N, ld);
   const int64_t nchunks = (N + chunk - 1) / chunk;
   if (chunk > INT32_MAX / 2 || V > INT32_MAX / 2) return GH_ERR_UNSUPPORTED;
-  const bool acc32 = a.accum == GH_ACCUM_FP32 && nchunks > 1;
+  // fp32 accumulator: library scratch when several chunks must be summed before
+  // the single rounding, or the caller's fp32 output (dW32: no rounding here)
+  const bool out32 = a.dW32 != nullptr;
+  const bool acc32 = !out32 && a.accum == GH_ACCUM_FP32 && nchunks > 1;
   const bool pair = use_pairs();
   const int tile_m = pair ? sm100::GemmCfg<true>::kTileM : sm100::GemmCfg<false>::kTileM;
   const int sms = sm_count();
@@ -346,7 +375,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const unsigned long long* n_valid = a.n_total ? a.n_total : counter;
   float* row_loss = reinterpret_cast<float*>(base + off_rows);
   uint16_t* L = reinterpret_cast<uint16_t*>(base + off_buf);
-  float* acc = acc32 ? reinterpret_cast<float*>(base + off_acc) : nullptr;
+  float* acc = acc32 ? reinterpret_cast<float*>(base + off_acc) : out32 ? a.dW32 : nullptr;
   float* ws = dx_splits > 1 ? reinterpret_cast<float*>(base + off_ws) : nullptr;
   float2* stats = fused ? reinterpret_cast<float2*>(base + off_stats) : nullptr;
   float* x_target = fused ? reinterpret_cast<float*>(base + off_xt) : nullptr;
@@ -372,7 +401,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   CUtensorMap tm_w_k, tm_w_n, tm_dw_out, tm_acc, tm_ws;
   if (st == GH_OK &&
       (!make_tmap(&tm_w_k, W, D, V, D * 2, pair ? sm100::GemmCfg<true>::kBRows : sm100::GemmCfg<false>::kBRows) || !make_tmap(&tm_w_n, W, D, V, D * 2, 64) ||
-       !make_out_bf16(&tm_dw_out, dW, D, V, D) || (acc32 && !make_out_f32(&tm_acc, acc, D, V, D)) ||
+       (!out32 && !make_out_bf16(&tm_dw_out, dW, D, V, D)) || ((acc32 || out32) && !make_out_f32(&tm_acc, acc, D, V, D)) ||
        (ws && !make_out_f32(&tm_ws, ws, D, dx_splits * rows_pad, D))))
     st = GH_ERR_CUDA;
 
@@ -485,8 +514,16 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     sm100::GemmArgs g4 = gemm_args(static_cast<int>(V), static_cast<int>(D), rows, 0, sm100::kEpiStoreBf16, pair);
     g4.out = dW;
     g4.ld_out = D;
+    // dW reads P and the (scaled) inputs, which the dX GEMM before it waited
+    // for before letting dependents launch, and nothing dX writes: its tiles
+    // start as dX's CTAs retire; it completes after dX, so the next chunk's
+    // logits GEMM cannot overwrite P while dX reads it.
+    g4.defer_wait = 1;
     const CUtensorMap* out4 = &tm_dw_out;
-    if (a.accum == GH_ACCUM_FP32) {
+    if (out32) {
+      g4.epi = c == 0 ? sm100::kEpiStoreF32 : sm100::kEpiAddF32;
+      out4 = &tm_acc;
+    } else if (a.accum == GH_ACCUM_FP32) {
       if (acc32 && c + 1 < nchunks) {
         g4.epi = c == 0 ? sm100::kEpiStoreF32 : sm100::kEpiAddF32;
         out4 = &tm_acc;

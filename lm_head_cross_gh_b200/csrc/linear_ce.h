@@ -24,7 +24,12 @@ struct LinearCeArgs {
   gh_chunk_loss_fn loss_fn;  // null: cross-entropy; else the caller's loss per chunk
   void* loss_ctx;
   const unsigned long long* n_total;  // non-null: the mean divides by this count (all shards)
+  float* dW32;             // non-null (fp32 accumulation only): grad_weight is returned here as the
+                           // unrounded fp32 sum over the chunks, [V, D], and dW is not written
 };
+
+// out[i] = bf16(src[i]) (round to nearest even), n elements.
+gh_status_t cast_f32_bf16_launch(const float* src, void* out, int64_t n, cudaStream_t stream);
 
 gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream);
 

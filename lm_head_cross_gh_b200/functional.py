@@ -22,7 +22,8 @@ Data parallel (one process per GPU, a batch split over the ranks of a
   return the whole batch's loss on every rank and, in backward, this rank's share
   of its gradients: the valid-token counts are summed over the ranks first (one
   int64 all-reduce), every shard divides by that total, the shards' losses are
-  summed (one scalar all-reduce) and so are the weight gradients.
+  summed (one scalar all-reduce) and so are the weight gradients (fp32
+  accumulators summed in fp32 and rounded once, for fp32 accumulation).
 """
 from __future__ import annotations
 
@@ -192,10 +193,19 @@ class _DPLinearCE(torch.autograd.Function):
     def forward(ctx, inputs, weight, target, ignore_index, reduction, z, accum, group, ops):
         t = target.contiguous()
         n = _all_reduce_sum(ops.gh_count_valid(t, weight.shape[0], ignore_index), group)
-        loss, dX, dW = ops.gh_linear_ce_shard(inputs.contiguous(), weight.contiguous(), t, n, ignore_index,
-                                              reduction, z, 0, accum)
+        if accum == "fp32":
+            # every shard's fp32 accumulator is summed in fp32 and the batch's sum
+            # is rounded to the weight dtype once
+            loss, dX, dW32 = ops.gh_linear_ce_shard_f32(inputs.contiguous(), weight.contiguous(), t, n,
+                                                        ignore_index, reduction, z, 0)
+            dW = ops.gh_cast_f32_to_bf16(_all_reduce_sum(dW32, group))
+        else:
+            # "weight": each shard rounds between its chunks; the shards' sums are
+            # added in the weight dtype
+            loss, dX, dW = ops.gh_linear_ce_shard(inputs.contiguous(), weight.contiguous(), t, n, ignore_index,
+                                                  reduction, z, 0, accum)
+            dW = _all_reduce_sum(dW, group)
         loss = _all_reduce_sum(loss, group)
-        dW = _all_reduce_sum(dW, group)
         ctx.save_for_backward(dX, dW)
         return loss
 
@@ -211,6 +221,7 @@ def data_parallel_chunked_linear_cross_entropy(inputs, weight, target, ignore_in
                                                grad_weight_accum_dtype: str = "fp32", group=None, ops=None):
     """``chunked_linear_cross_entropy`` of the whole batch whose rows ``inputs`` /
     ``target`` this rank holds, with the weight replicated: the weight gradient
-    is summed over the ranks (in the weight dtype)."""
+    is summed over the ranks, in fp32 and rounded once for
+    ``grad_weight_accum_dtype="fp32"``, in the weight dtype for ``"weight"``."""
     return _DPLinearCE.apply(inputs, weight, target, ignore_index, reduction, float(z_loss_multiplier),
                              grad_weight_accum_dtype, group, _ops(ops))

@@ -50,6 +50,17 @@ class _HostOps:
         loss, G = cls.gh_ce_fwd_bwd_shard(X @ W.T, t, n, ii, reduction, z)
         return loss, G @ W, G.T @ X
 
+    @classmethod
+    def gh_linear_ce_shard_f32(cls, X, W, t, n, ii, reduction, z, chunk):
+        """bf16 inputs; the shard's weight gradient as an unrounded fp32 sum."""
+        X64, W64 = X.double(), W.double()
+        loss, G = cls.gh_ce_fwd_bwd_shard(X64 @ W64.T, t, n, ii, reduction, z)
+        return loss.float(), (G @ W64).to(X.dtype), (G.T @ X64).float()
+
+    @staticmethod
+    def gh_cast_f32_to_bf16(src):
+        return src.to(torch.bfloat16)
+
 
 def _batch(seed=0, N=24, D=6, V=17):
     g = torch.Generator().manual_seed(seed)
@@ -75,7 +86,8 @@ def _rank_main(rank, world, port, out):
     # linear CE with a replicated weight
     Xs = X[rows].clone().requires_grad_(True)
     Wr = W.clone().requires_grad_(True)
-    lin = GF.data_parallel_chunked_linear_cross_entropy(Xs, Wr, t[rows], -100, "mean", 1e-3, ops=_HostOps)
+    lin = GF.data_parallel_chunked_linear_cross_entropy(Xs, Wr, t[rows], -100, "mean", 1e-3,
+                                                        grad_weight_accum_dtype="weight", ops=_HostOps)
     lin.backward()
     out.put((rank, loss.item(), logits.grad, lin.item(), Xs.grad, Wr.grad))
     dist.barrier()
@@ -105,3 +117,49 @@ def test_two_gloo_ranks_data_parallel_cross_entropy():
         assert lin == pytest.approx(lf.item(), rel=1e-12)
         assert torch.allclose(gx, (Gf @ W)[rows], rtol=1e-10, atol=1e-13)
         assert torch.allclose(gw, Gf.T @ X, rtol=1e-10, atol=1e-13)
+
+
+def _rank_main_fp32(rank, world, port, out):
+    """bf16 inputs and weight with fp32 weight-gradient accumulation: each rank's
+    fp32 accumulator is all-reduced in fp32 and the sum rounded once."""
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+    from lm_head_cross_gh_b200 import functional as GF
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    X, W, t = _batch(seed=3, N=40, D=16, V=33)
+    rows = slice(rank * 20, (rank + 1) * 20)
+    Xs = X[rows].to(torch.bfloat16).requires_grad_(True)
+    Wr = W.to(torch.bfloat16).requires_grad_(True)
+    lin = GF.data_parallel_chunked_linear_cross_entropy(Xs, Wr, t[rows], -100, "mean", 1e-3,
+                                                        grad_weight_accum_dtype="fp32", ops=_HostOps)
+    lin.backward()
+    out.put((rank, lin.item(), Wr.grad))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_fp32_weight_gradient_is_rounded_once():
+    """'fp32' accumulation across ranks: the weight gradient every rank holds is
+    bf16(fp32 partial of rank 0 + fp32 partial of rank 1), one rounding of the
+    fp32 sum, not a sum of bf16-rounded partials."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_fp32, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=180) for _ in procs), key=lambda r: r[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    X, W, t = _batch(seed=3, N=40, D=16, V=33)
+    Xb, Wb = X.to(torch.bfloat16), W.to(torch.bfloat16)
+    n = torch.tensor(int((t != -100).sum()))
+    parts = [_HostOps.gh_linear_ce_shard_f32(Xb[r * 20:(r + 1) * 20], Wb, t[r * 20:(r + 1) * 20], n, -100, "mean",
+                                             1e-3, 0)[2] for r in range(2)]
+    once = (parts[0] + parts[1]).to(torch.bfloat16)
+    twice = (parts[0].to(torch.bfloat16) + parts[1].to(torch.bfloat16))
+    assert not torch.equal(once, twice)  # the two readings differ on this batch
+    for rank, lin, gw in res:
+        assert gw.dtype == torch.bfloat16
+        assert torch.equal(gw, once), rank

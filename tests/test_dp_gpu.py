@@ -3,7 +3,9 @@
 gh_ce_fwd_bwd_shard / gh_linear_ce_shard divide the mean by a total count the
 caller passes; with a total of twice the local count the loss and gradients
 are the oracle's for scale 1 / (2 n_valid).  With the local count they are
-bitwise those of gh_ce_fwd_bwd / gh_linear_ce.  The data-parallel functional
+bitwise those of gh_ce_fwd_bwd / gh_linear_ce.  gh_linear_ce_shard_f32 returns
+the weight gradient's unrounded fp32 sum (rounded once by gh_cast_f32_to_bf16
+it is the bf16 entry point's).  The data-parallel functional
 wrappers on a one-rank NCCL group (the all-reduces are then identities) give
 the same results as the single-process functions.
 """
@@ -56,6 +58,41 @@ def test_linear_ce_shard_with_the_local_count_is_linear_ce(cuda_device):
     b = gh.gh_linear_ce(X, W, t, -100, "mean", 1e-4, 256, "fp32")
     torch.cuda.synchronize()
     assert a[0].item() == b[0].item() and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+
+
+@pytest.mark.parametrize("chunk", [256, 0])
+def test_linear_ce_shard_f32_returns_the_unrounded_weight_gradient(cuda_device, chunk):
+    """The fp32 shard entry point's weight gradient is the fp32 sum over the
+    chunks: against the oracle (scale 1 / (2 n_valid)), and rounded once it is
+    bitwise the bf16 shard entry point's."""
+    q = gh_synth.linear_ce_normal(700, 128, 3001, chunk=chunk, ignore_frac=0.05, w_sigma=0.05, z_loss=1e-4, seed=15)
+    X = torch.from_numpy(q.inputs.view(np.int16)).cuda().view(torch.bfloat16)
+    W = torch.from_numpy(q.weight.view(np.int16)).cuda().view(torch.bfloat16)
+    t = torch.from_numpy(q.targets).cuda()
+    n_local = int((q.targets != -100).sum())
+    total = torch.tensor(2 * n_local, dtype=torch.int64, device="cuda")
+    l32, dx32, dw32 = gh.gh_linear_ce_shard_f32(X, W, t, total, -100, "mean", 1e-4, chunk)
+    l16, dx16, dw16 = gh.gh_linear_ce_shard(X, W, t, total, -100, "mean", 1e-4, chunk, "fp32")
+    torch.cuda.synchronize()
+    assert dw32.dtype == torch.float32
+    assert l32.item() == l16.item() and torch.equal(dx32, dx16)
+    assert torch.equal(gh.gh_cast_f32_to_bf16(dw32), dw16)
+    Xd = gh_synth.bf16_to_f32(q.inputs).astype(np.float64)
+    Wd = gh_synth.bf16_to_f32(q.weight).astype(np.float64)
+    r = oracle.linear_cross_entropy(Xd, Wd, q.targets, -100, "sum", 1e-4, chunk, "fp32")
+    ref = r["grad_weight"] / (2 * n_local)   # "sum" scaled by the batch's mean factor
+    got = dw32.cpu().numpy().astype(np.float64)
+    assert np.linalg.norm(got - ref) <= 1e-2 * np.linalg.norm(ref)
+
+
+def test_cast_f32_to_bf16_rounds_to_nearest_even(cuda_device):
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn(100003, generator=g) * torch.exp(torch.randn(100003, generator=g) * 8)
+    x[:6] = torch.tensor([0.0, -0.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 3.0e38, -1.0e-40])
+    xd = x.cuda()
+    got = gh.gh_cast_f32_to_bf16(xd)
+    torch.cuda.synchronize()
+    assert torch.equal(got.view(torch.int16), xd.to(torch.bfloat16).view(torch.int16))
 
 
 def _free_port():
