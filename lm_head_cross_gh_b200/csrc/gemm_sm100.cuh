@@ -109,7 +109,12 @@ struct GemmArgs {
   const float* split_ws;
   uint16_t* split_out;
   int64_t split_ld;
-  int* split_count;        // one counter per (tile, CTA of the pair, 32-row slice), 0 between launches
+  int* split_count;        // one counter per (tile, CTA of the pair, 32-row slice)
+  // 0: the last split to finish a slice sums it (counters back to 0 after each
+  // launch).  > 0: every unit of the launch is resident at once, and each split
+  // waits (bounded) until the slice's counter reaches split_target, then sums
+  // every k_splits-th row of the slice (counters only grow within a call).
+  int split_target;
   // kEpiAccToBf16
   const float* acc;
   int64_t acc_ld;
@@ -845,27 +850,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) bulk_wait_all();
         __syncwarp();
         const int cidx = ((mb * g.tiles_n + nb) * (PAIR ? 2 : 1) + static_cast<int>(rank)) * 4 + q;
-        int last = 0;
+        // rows r0, r0 + rstep, ... of the slice are summed by this warp
+        int r0 = 0, rstep = 1;
+        int go = 0;
         if (lane == 0) {
           __threadfence();
-          last = atomicAdd(&g.split_count[cidx], 1) == g.k_splits - 1;
+          const int before = atomicAdd(&g.split_count[cidx], 1);
+          if (g.split_target > 0) {
+            // every split's warp waits for the others, then takes its share of the rows
+            const volatile int* cnt = &g.split_count[cidx];
+            const uint64_t t0 = global_timer_ns();
+            go = 1;
+            while (*cnt < g.split_target) {
+              if (global_timer_ns() - t0 > wait_limit_ns()) {
+                record_status(GH_ERR_TIMEOUT);
+                go = 0;
+                break;
+              }
+              __nanosleep(64);
+            }
+          } else {
+            go = before == g.k_splits - 1;  // the last split sums the whole slice
+            if (go) g.split_count[cidx] = 0;
+          }
         }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (g.split_target > 0) {
+          r0 = ks;
+          rstep = g.k_splits;
+        }
+        if (go) {
           __threadfence();  // every split's partial of this slice is visible
-          if (lane == 0) g.split_count[cidx] = 0;
           const int col = nb * kBN + 8 * lane;  // lanes across the row: coalesced 32-byte reads
           if (col < g.N) {
             // 2 rows at a time with every split's loads issued before the adds
 #pragma unroll 1
-            for (int r0 = 0; r0 < 32; r0 += 2) {
+            for (int r = r0; r < 32; r += 2 * rstep) {
               float4 u[kMaxSplits][2][2];
 #pragma unroll
               for (int sp = 0; sp < kMaxSplits; ++sp) {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                  const int rr = rbase + r0 + i;
-                  if (sp < g.k_splits && rr < g.M) {
+                  const int rr = rbase + r + i * rstep;
+                  if (sp < g.k_splits && r + i * rstep < 32 && rr < g.M) {
                     const float* p = g.split_ws + (static_cast<int64_t>(sp) * g.split_rows + rr) * g.N + col;
                     u[sp][i][0] = __ldcg(reinterpret_cast<const float4*>(p));
                     u[sp][i][1] = __ldcg(reinterpret_cast<const float4*>(p + 4));
@@ -874,8 +901,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
 #pragma unroll
               for (int i = 0; i < 2; ++i) {
-                const int rr = rbase + r0 + i;
-                if (rr >= g.M) break;
+                const int rr = rbase + r + i * rstep;
+                if (r + i * rstep >= 32 || rr >= g.M) break;
                 float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int sp = 0; sp < kMaxSplits; ++sp) {

@@ -269,20 +269,22 @@ sm100::GemmArgs gemm_args(int M, int N, int K, int m_fastest, int epi, bool pair
   return g;
 }
 
-// K splits for a GEMM whose output tiles would leave SMs idle: the split count
-// that minimises (waves of work units) x (K steps per unit), each unit at
-// least 16 K steps long; the smallest such count on ties.
-int choose_splits(int tiles, int num_kb, int sms) {
-  if (tiles >= sms) return 1;
+// K splits for a long-K GEMM: the split count (at most max_splits, each split
+// at least 16 K steps) that minimises (waves of work units) x (K steps per
+// unit), when that saves at least 3% over no split.  It fills SMs that the
+// output tiles alone would leave idle, and evens out a last wave of tiles
+// that would run part-empty.
+int choose_splits(int tiles, int num_kb, int units, int max_splits) {
   int best = 1;
-  int64_t best_cost = static_cast<int64_t>(num_kb);
-  const int smax = std::max(1, num_kb / 16);
+  const int64_t base = (static_cast<int64_t>(tiles) + units - 1) / units * num_kb;
+  int64_t best_cost = base;
+  const int smax = std::min(max_splits, std::max(1, num_kb / 16));
   for (int sp = 2; sp <= smax; ++sp) {
     const int per = (num_kb + sp - 1) / sp;
     const int used = (num_kb + per - 1) / per;
-    const int64_t waves = (static_cast<int64_t>(tiles) * used + sms - 1) / sms;
+    const int64_t waves = (static_cast<int64_t>(tiles) * used + units - 1) / units;
     const int64_t cost = waves * per;
-    if (cost < best_cost) {
+    if (cost < best_cost && cost * 100 <= base * 97) {
       best_cost = cost;
       best = used;
     }
@@ -336,7 +338,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const int tiles_m_max = static_cast<int>((chunk + tile_m - 1) / tile_m);
   const int dx_num_kb = static_cast<int>((V + sm100::kBK - 1) / sm100::kBK);
   const int dx_tiles_max = tiles_m_max * static_cast<int>((D + sm100::kBN - 1) / sm100::kBN);
-  const int dx_splits = std::min(sm100::kMaxSplits, choose_splits(dx_tiles_max, dx_num_kb, units));
+  const int dx_splits = choose_splits(dx_tiles_max, dx_num_kb, units, sm100::kMaxSplits);
   const int64_t rows_pad = static_cast<int64_t>(tiles_m_max) * tile_m;
 
   const bool custom = a.loss_fn != nullptr;
@@ -405,6 +407,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
        (ws && !make_out_f32(&tm_ws, ws, D, dx_splits * rows_pad, D))))
     st = GH_ERR_CUDA;
 
+  int split_base = 0;  // arrivals per split counter so far in this call (cooperative split sums)
   for (int64_t c = 0; c < nchunks && st == GH_OK; ++c) {
     const int64_t c0 = c * chunk;
     const int rows = static_cast<int>(std::min<int64_t>(chunk, N - c0));
@@ -491,7 +494,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     // 3: dX_c = G_c W (K split into fp32 partials when the tiles alone leave SMs idle)
     sm100::GemmArgs g3 = gemm_args(rows, static_cast<int>(D), static_cast<int>(V), 1, sm100::kEpiStoreBf16, pair);
     g3.row_scale = alpha;  // null on the plain path
-    const int splits = choose_splits(g3.tiles_m * g3.tiles_n, g3.num_kb, units);
+    const int splits = choose_splits(g3.tiles_m * g3.tiles_n, g3.num_kb, units, sm100::kMaxSplits);
     if (splits > 1 && ws) {
       g3.k_splits = std::min(splits, dx_splits);
       g3.kb_per_split = (g3.num_kb + g3.k_splits - 1) / g3.k_splits;
@@ -503,6 +506,11 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       g3.split_out = dX + c0 * D;
       g3.split_ld = D;
       g3.split_count = split_count;
+      if (g3.tiles_m * g3.tiles_n * g3.k_splits <= units) {
+        // every unit has its own SM (pair) at once: the splits share the sums
+        split_base += g3.k_splits;
+        g3.split_target = split_base;
+      }
       st = launch_gemm<false, true>(tm_l_k, tm_w_n, tm_ws, g3, pair, GH_KERNEL_DX_GEMM, stream);
       if (st != GH_OK) break;
     } else {

@@ -73,6 +73,7 @@ def test_small_three_ragged_chunks(cuda_device, accum, reduction, z):
     (200, 72, 300, 0),        # D not a multiple of 64, default chunk
     (640, 256, 2049, 384),    # several full N tiles, V just past a tile
     (1000, 768, 5003, 384),   # GPT-2 width, ragged everything
+    (4096, 1280, 4099, 0),    # dX tiles past one wave: K split with more units than SMs
 ])
 def test_shapes(cuda_device, N, D, V, chunk):
     p = gh_synth.linear_ce_normal(N, D, V, chunk=chunk, ignore_frac=0.1, x_sigma=1.0, w_sigma=0.5 / np.sqrt(D),
