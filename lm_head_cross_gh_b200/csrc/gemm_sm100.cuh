@@ -43,7 +43,7 @@ constexpr int kBM = 128;                      // accumulator rows of one CTA (TM
 constexpr int kBN = 256;                      // accumulator columns (one tcgen05.mma N)
 constexpr int kBK = 64;                       // one 128-byte swizzle row of bf16
 constexpr int kABytes = kBM * kBK * 2;        // 16 KiB
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;  // producer, MMA, 4 epilogue warps, second producer
 constexpr int kTmemCols = 2 * kBN;            // two accumulators
 constexpr int kStageOutBytes = 4096;          // one epilogue staging buffer: 32 rows x 128 bytes
 constexpr int kOutBytes = 4 * 2 * kStageOutBytes;  // 4 epilogue warps x 2 buffers
@@ -64,6 +64,7 @@ struct GemmCfg {
 };
 constexpr int kGemmSmem = GemmCfg<false>::kSmem;
 constexpr int kMaxSplits = 4;  // K splits a tile may be cut into when they are summed in the kernel
+constexpr int kProducers = 2;  // TMA producer warps (warps 0 and 6)
 static_assert(GemmCfg<true>::kSmem <= 232448 && GemmCfg<false>::kSmem <= 232448, "shared memory per CTA");
 
 // Epilogue modes (what happens to the fp32 tile).  The first three go out
@@ -416,37 +417,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     kb1 = min(g.num_kb, kb0 + g.kb_per_split);
   };
 
-  if (warp == 0) {
-    // ---------------- TMA producer (both CTAs of a pair: each loads its halves) ----------------
+  if (warp == 0 || warp == 6) {
+    // ---------------- TMA producers (both CTAs of a pair: each loads its halves) ----------------
+    // Warp 0 and warp 6 each take every other stage load of this CTA's sequence
+    // of (tile, K step) items (one issuing thread alone is slower than the loads
+    // it issues); kStages is even, so a stage always has the same producer.
+    static_assert(kStages % kProducers == 0, "stages per producer");
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0;  // stages this producer armed
-      bool run = true;
-      for (int tile = unit; tile < num_tiles_run && run; tile += units) {
-        int mb, nb, ks, kb0, kb1;
+      const int pw = warp == 0 ? 0 : 1;  // this producer's items: pw, pw + kProducers, ...
+      int tile = unit, mb = 0, nb = 0, ks = 0, kb0 = 0, kb1 = 0, kb = 0;
+      bool have = tile < num_tiles_run;
+      if (have) {
         tile_coords(tile, mb, nb, ks);
         kb_range(ks, kb0, kb1);
-        const int m0 = mb * C::kTileM + static_cast<int>(rank) * kBM;
-        const int n0 = nb * kBN + static_cast<int>(rank) * C::kBRows;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!wait_or_abort<PAIR>(&empty[stage], phase ^ 1, abort_flag)) {
-            run = false;
-            break;
-          }
+        kb = kb0;
+      }
+      auto next_item = [&]() -> bool {  // the next (tile, K step) of this CTA's sequence
+        if (++kb < kb1) return true;
+        tile += units;
+        if (tile >= num_tiles_run) return false;
+        tile_coords(tile, mb, nb, ks);
+        kb_range(ks, kb0, kb1);
+        kb = kb0;
+        return kb < kb1;
+      };
+      for (int i = 0; i < pw && have; ++i) have = next_item();
+      uint32_t item = static_cast<uint32_t>(pw);  // linear index of this producer's next load
+      uint32_t done = 0;                          // loads this producer issued
+      while (have) {
+        const int stage = static_cast<int>(item % kStages);
+        const uint32_t phase = (item / kStages) & 1u;
+        if (!wait_or_abort<PAIR>(&empty[stage], phase ^ 1, abort_flag)) break;
+        const bool withhold =
+            g.withhold_plus1 != 0 && unit == 0 && leader && item + 1 == static_cast<uint32_t>(g.withhold_plus1);
+        if (!withhold) {
+          // (withheld, for a test of the failure path: this stage's barrier is
+          // never armed, so the MMA issuer's bounded wait for it runs out)
           uint8_t* sa = stage_base + stage * kStageBytes;
           uint8_t* sb = sa + kABytes;
           const int k0 = kb * kBK;
-          if (g.withhold_plus1 != 0 && unit == 0 && leader && issued + 1 == static_cast<uint32_t>(g.withhold_plus1)) {
-            // test of the failure path: this stage's barrier is never armed,
-            // so the MMA issuer's bounded wait for it runs out
-            ++issued;
-            if (++stage == kStages) {
-              stage = 0;
-              phase ^= 1;
-            }
-            continue;
-          }
+          const int m0 = mb * C::kTileM + static_cast<int>(rank) * kBM;
+          const int n0 = nb * kBN + static_cast<int>(rank) * C::kBRows;
           auto load = [&](void* dst, const CUtensorMap* map, int x, int y) {
             if constexpr (PAIR) {
               if (!leader) {
@@ -470,12 +481,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
             load(sb, &tma_b, k0, n0);
           }
-          ++issued;
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
         }
+        ++done;
+        item += kProducers;
+        for (int i = 0; i < kProducers && have; ++i) have = next_item();
       }
       if (*abort_flag) {
         // copies still in flight land before the CTA exits: the leader's stage
@@ -483,7 +492,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // cannot see its own and waits out a fixed, generous interval instead
         if (leader) {
           const uint64_t t0 = global_timer_ns();
-          for (uint32_t n = (issued > kStages ? issued - kStages : 0); n < issued; ++n) {
+          for (uint32_t d = 0; d < done && d < static_cast<uint32_t>(kStages / kProducers); ++d) {
+            const uint32_t n = item - kProducers * (d + 1);  // this producer's last loads
             const uint32_t a = smem_u32(&full[n % kStages]);
             while (!mbar_try_wait(a, (n / kStages) & 1, 20000u) && global_timer_ns() - t0 < wait_limit_ns()) {
             }
