@@ -48,7 +48,10 @@ METRIC = "CE tokens/s and HBM GB/s; linear-CE tokens/s and TFLOP/s vs bf16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 CE_WORKLOADS = {"ce_gpt2": "ce_gpt2", "ce_large_vocab": "ce_large_vocab", "ce_small": "ce_small"}
-LINEAR_WORKLOADS = {"linear_ce_gpt2": "linear_ce_gpt2", "linear_ce_llama3_8b": "linear_ce_llama3_8b"}
+# bench name -> (generator in gh_synth, grad_weight accumulation or None for the generator's own)
+LINEAR_WORKLOADS = {"linear_ce_gpt2": ("linear_ce_gpt2", None),
+                    "linear_ce_gpt2_weight_accum": ("linear_ce_gpt2", "weight"),
+                    "linear_ce_llama3_8b": ("linear_ce_llama3_8b", None)}
 
 
 def peaks():
@@ -265,7 +268,11 @@ def make_ce(name, seed):
 
 def make_linear(name, seed):
     import gh_synth
-    p = getattr(gh_synth, LINEAR_WORKLOADS[name])(seed=seed)
+    gen, accum = LINEAR_WORKLOADS[name]
+    p = getattr(gh_synth, gen)(seed=seed)
+    if accum is not None and accum != p.accum:
+        p.accum = accum
+        p.name += f"_{accum}_accum"
     if ROWS:
         p.inputs = p.inputs[:ROWS].copy()
         p.targets = p.targets[:ROWS].copy()
@@ -598,6 +605,7 @@ def run_oracle_timing(case, budget_rows, reps=1):
 
 # Oracle rows per host thread in one timing sample (linear-CE: per sample, BLAS-threaded).
 ORACLE_ROWS = {"ce_gpt2": 1024, "ce_large_vocab": 64, "ce_small": 64, "linear_ce_gpt2": 512,
+               "linear_ce_gpt2_weight_accum": 512,
                "linear_ce_llama3_8b": 32}
 
 
@@ -668,8 +676,8 @@ def measure(case, dist, steps, warmup, pk, pk_kind):
 
 
 # Workloads the default CE line also carries (name, steps cap).
-EXTRA_WORKLOADS = (("linear_ce", "linear_ce_gpt2", 20), ("linear_ce_llama3_8b", "linear_ce_llama3_8b", 3),
-                   ("ce_large_vocab", "ce_large_vocab", 20))
+EXTRA_WORKLOADS = (("linear_ce", "linear_ce_gpt2", 20), ("linear_ce_weight_accum", "linear_ce_gpt2_weight_accum", 20),
+                   ("linear_ce_llama3_8b", "linear_ce_llama3_8b", 3), ("ce_large_vocab", "ce_large_vocab", 20))
 
 
 def make_case(name, seed, dev, op="fwd_bwd"):

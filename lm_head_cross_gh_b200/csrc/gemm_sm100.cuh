@@ -74,7 +74,7 @@ enum GemmEpi : int {
   kEpiStoreBf16 = 0,  // out(bf16) = tile                       TMA store
   kEpiStoreF32 = 1,   // out(f32)  = tile                       TMA store
   kEpiAddF32 = 2,     // out(f32) += tile                       TMA reduce-add (in L2)
-  kEpiBf16Add = 3,    // out = bf16(float(out) + tile), direct loads and stores (bf16 accumulator)
+  kEpiBf16Add = 3,    // out(bf16) = bf16(out + tile)          TMA load, add in place, TMA store
   kEpiCeExp = 4,      // logits tile of the fused cross-entropy: out(bf16) = exp(tile - R_row)
                       // (0 for ignored rows), plus per (row, column tile) sum and max
   kEpiAccToBf16 = 5   // out(bf16) = bf16(acc + tile), acc an fp32 [M, acc_ld] array   TMA store
@@ -88,9 +88,6 @@ struct GemmArgs {
   int split_rows;       // row offset in the output map between K splits
   int m_fastest;        // tile order: consecutive tiles share the B tile (1) or the A tile (0)
   int epi;
-  void* out;            // kEpiBf16Add only: bf16 [M, ld_out]
-  int64_t ld_out;
-  int m_limit, n_limit; // kEpiBf16Add only: rows / columns stored (n_limit a multiple of 8)
   // kEpiStoreBf16 / kEpiStoreF32: when non-null, output row r (of the M rows)
   // is multiplied by row_scale[r] before it is stored.
   const float* row_scale;
@@ -352,7 +349,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tmem_full = empty + kStages;
   uint64_t* tmem_empty = tmem_full + 2;
   uint64_t* mma_done = tmem_empty + 2;
-  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* epi_bar = mma_done + 1;  // kEpiBf16Add: one per epilogue staging buffer
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(epi_bar + 8);
+  static_assert((2 * kStages + 2 + 2 + 1 + 8) * 8 + 8 <= 256, "barriers, TMEM address and abort flag");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -373,11 +372,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tmem_empty[b], PAIR ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
     }
     mbar_init(mma_done, 1);
+    for (int b = 0; b < 8; ++b) mbar_init(&epi_bar[b], 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tma_a);
     prefetch_tmap(&tma_b);
-    if (g.epi != kEpiBf16Add) prefetch_tmap(&tma_out);
+    prefetch_tmap(&tma_out);
   }
   if (warp == 1) {
     tmem_alloc<PAIR>(tmem_base_slot, kTmemCols);
@@ -819,32 +819,72 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ++nstore;
         }
       } else if (kDw) {
-        // kEpiBf16Add: accumulate into the bf16 output with plain loads and stores
-        const bool row_ok = row < g.m_limit;
-#pragma unroll 1
-        for (int cc = 0; cc < kBN; cc += 32) {
-          uint32_t v[32];
-          tmem_ld32(t_row + cc, v);
-          tmem_ld_wait(v);
-          const int col0 = nb * kBN + cc;
-          if (!row_ok || col0 >= g.n_limit) continue;
-          const int ncols = min(32, g.n_limit - col0);  // a multiple of 8
-          uint16_t* o = reinterpret_cast<uint16_t*>(g.out) + static_cast<int64_t>(row) * g.ld_out + col0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j * 8 >= ncols) break;
-            const uint4 prev = *reinterpret_cast<const uint4*>(o + j * 8);
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[j * 8 + e]);
-            f[0] += bf16_lo(prev.x); f[1] += bf16_hi(prev.x);
-            f[2] += bf16_lo(prev.y); f[3] += bf16_hi(prev.y);
-            f[4] += bf16_lo(prev.z); f[5] += bf16_hi(prev.z);
-            f[6] += bf16_lo(prev.w); f[7] += bf16_hi(prev.w);
-            *reinterpret_cast<uint4*>(o + j * 8) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                                              pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+        // kEpiBf16Add: each 64-column slice of the warp's 32 output rows comes
+        // in by TMA (zeros outside the map) into a staging buffer, gets the
+        // tile added in place, rounded once to bf16, and goes back out by TMA
+        // (clipped outside the map).  The next slice's load flies while this
+        // slice is added.
+        auto issue = [&](int n, int x) {  // the warp's n-th slice, into buffer n & 1
+          if (lane == 0) {
+            uint64_t* bar = &epi_bar[2 * q + (n & 1)];
+            mbar_arrive_expect_tx(bar, kStageOutBytes);
+            tma_load_2d(my_stage + (n & 1) * kStageOutBytes, &tma_out, bar, x, y);
           }
+        };
+        // a buffer is free once the store that used it has read it: two
+        // slices back for the first slice, one back for the next
+        if (lane == 0) bulk_wait_read_1();
+        __syncwarp();
+        issue(nstore, nb * kBN);
+        bool ok = true;
+#pragma unroll 1
+        for (int cs = 0; cs < kBN; cs += 64) {
+          const int n = nstore;
+          const bool next = cs + 64 < kBN;
+          if (next) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+            issue(n + 1, nb * kBN + cs + 64);
+          }
+          uint32_t v0[32], v1[32];
+          tmem_ld32(t_row + cs, v0);
+          tmem_ld32(t_row + cs + 32, v1);
+          tmem_ld_wait(v0, v1);
+          ok = __all_sync(0xffffffffu, wait_or_abort<false>(&epi_bar[2 * q + (n & 1)], (n >> 1) & 1, abort_flag));
+          if (!ok) {
+            // the loads this warp issued land before the CTA exits
+            if (lane == 0) {
+              const uint64_t t0 = global_timer_ns();
+              for (int m = n; m <= n + (next ? 1 : 0); ++m) {
+                const uint32_t a = smem_u32(&epi_bar[2 * q + (m & 1)]);
+                while (!mbar_try_wait(a, (m >> 1) & 1, 20000u) && global_timer_ns() - t0 < wait_limit_ns()) {
+                }
+              }
+            }
+            __syncwarp();
+            break;
+          }
+          uint8_t* buf = my_stage + (n & 1) * kStageOutBytes;
+          uint8_t* rowp = buf + lane * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4* p = reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4));
+            const uint4 prev = *p;
+            const uint32_t* t = c < 4 ? &v0[8 * c] : &v1[8 * (c - 4)];
+            *p = make_uint4(pack_bf16x2(bf16_lo(prev.x) + __uint_as_float(t[0]), bf16_hi(prev.x) + __uint_as_float(t[1])),
+                            pack_bf16x2(bf16_lo(prev.y) + __uint_as_float(t[2]), bf16_hi(prev.y) + __uint_as_float(t[3])),
+                            pack_bf16x2(bf16_lo(prev.z) + __uint_as_float(t[4]), bf16_hi(prev.z) + __uint_as_float(t[5])),
+                            pack_bf16x2(bf16_lo(prev.w) + __uint_as_float(t[6]), bf16_hi(prev.w) + __uint_as_float(t[7])));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_out, buf, nb * kBN + cs, y);
+            bulk_commit();
+          }
+          ++nstore;
         }
+        if (!ok) break;
       }
       // every TMEM load of this accumulator is complete: hand it back to the MMA
       // warp (of the pair's leader)

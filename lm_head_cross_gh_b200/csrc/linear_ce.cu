@@ -264,8 +264,6 @@ sm100::GemmArgs gemm_args(int M, int N, int K, int m_fastest, int epi, bool pair
   g.kb_per_split = g.num_kb;
   g.m_fastest = m_fastest;
   g.epi = epi;
-  g.m_limit = M;
-  g.n_limit = N;
   return g;
 }
 
@@ -520,8 +518,6 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
 
     // 4: dW (+)= G_c^T X_c
     sm100::GemmArgs g4 = gemm_args(static_cast<int>(V), static_cast<int>(D), rows, 0, sm100::kEpiStoreBf16, pair);
-    g4.out = dW;
-    g4.ld_out = D;
     // dW reads P and the (scaled) inputs, which the dX GEMM before it waited
     // for before letting dependents launch, and nothing dX writes: its tiles
     // start as dX's CTAs retire; it completes after dX, so the next chunk's
