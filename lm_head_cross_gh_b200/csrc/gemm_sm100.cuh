@@ -77,7 +77,7 @@ enum GemmEpi : int {
   kEpiBf16Add = 3,    // out(bf16) = bf16(out + tile)          TMA load, add in place, TMA store
   kEpiCeExp = 4,      // logits tile of the fused cross-entropy: out(bf16) = exp(tile - R_row)
                       // (0 for ignored rows), plus per (row, column tile) sum and max
-  kEpiAccToBf16 = 5   // out(bf16) = bf16(acc + tile), acc an fp32 [M, acc_ld] array   TMA store
+  kEpiAccToBf16 = 5   // out(bf16) = bf16(acc + tile), acc the fp32 array of `tma_aux`   TMA loads and store
 };
 
 struct GemmArgs {
@@ -113,9 +113,6 @@ struct GemmArgs {
   // waits (bounded) until the slice's counter reaches split_target, then sums
   // every k_splits-th row of the slice (counters only grow within a call).
   int split_target;
-  // kEpiAccToBf16
-  const float* acc;
-  int64_t acc_ld;
   // failure-path tests: 1 + the stage of unit 0's first tile whose loads the
   // producer leaves out (0: none)
   int withhold_plus1;
@@ -331,7 +328,8 @@ __device__ __forceinline__ void sleep_ns_bounded(uint64_t ns) {
 template <bool A_MN, bool B_MN, bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                     const __grid_constant__ CUtensorMap tma_out, GemmArgs g) {
+                     const __grid_constant__ CUtensorMap tma_out, const __grid_constant__ CUtensorMap tma_aux,
+                     GemmArgs g) {
   using C = GemmCfg<PAIR>;
   // Each operand layout serves one contraction, so each instantiation keeps
   // only the epilogues that contraction uses (fewer live registers).
@@ -378,6 +376,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     prefetch_tmap(&tma_a);
     prefetch_tmap(&tma_b);
     prefetch_tmap(&tma_out);
+    if (g.epi == kEpiAccToBf16) prefetch_tmap(&tma_aux);
   }
   if (warp == 1) {
     tmem_alloc<PAIR>(tmem_base_slot, kTmemCols);
@@ -757,35 +756,65 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           g.stats[static_cast<int64_t>(nb) * g.stats_ld + row] =
               make_float2((s0 + s1) + (s2 + s3), fmaxf(m0, m1));
       } else if (kDw && g.epi == kEpiAccToBf16) {
-        // the fp32 accumulator's rows plus this tile, rounded once to bf16
+        // Each 64-column slice: the fp32 accumulator's 32 rows come in by TMA
+        // (two 32-column boxes, one per staging buffer, zeros outside the
+        // map), the tile is added, the sum rounded once to bf16 and stored by
+        // TMA from the first buffer (clipped outside the map).
 #pragma unroll 1
         for (int cs = 0; cs < kBN; cs += 64) {
+          const int n = nstore;
+          uint64_t* bar = &epi_bar[2 * q];
+          if (lane == 0) {
+            bulk_wait_read_all();  // the previous slice's store has read the first buffer
+            mbar_arrive_expect_tx(bar, 2 * kStageOutBytes);
+            tma_load_2d(my_stage, &tma_aux, bar, nb * kBN + cs, y);
+            tma_load_2d(my_stage + kStageOutBytes, &tma_aux, bar, nb * kBN + cs + 32, y);
+          }
+          __syncwarp();
           uint32_t v0[32], v1[32];
           tmem_ld32(t_row + cs, v0);
           tmem_ld32(t_row + cs + 32, v1);
           tmem_ld_wait(v0, v1);
-          const int col = nb * kBN + cs;
-          if (row < g.M) {
-            const float* a = g.acc + static_cast<int64_t>(row) * g.acc_ld + col;
-#pragma unroll
-            for (int j = 0; j < 64; j += 4) {
-              if (col + j < g.N) {  // N is a multiple of 8
-                const float4 p = __ldcs(reinterpret_cast<const float4*>(a + j));
-                uint32_t* w = j < 32 ? &v0[j] : &v1[j - 32];
-                w[0] = __float_as_uint(__uint_as_float(w[0]) + p.x);
-                w[1] = __float_as_uint(__uint_as_float(w[1]) + p.y);
-                w[2] = __float_as_uint(__uint_as_float(w[2]) + p.z);
-                w[3] = __float_as_uint(__uint_as_float(w[3]) + p.w);
+          if (!__all_sync(0xffffffffu, wait_or_abort<false>(bar, n & 1, abort_flag))) {
+            if (lane == 0) {  // the two loads land before the CTA exits
+              const uint64_t t0 = global_timer_ns();
+              while (!mbar_try_wait(smem_u32(bar), n & 1, 20000u) && global_timer_ns() - t0 < wait_limit_ns()) {
               }
             }
+            __syncwarp();
+            break;
           }
-          uint32_t pk[32];
+          uint8_t* rowp = my_stage + lane * 128;
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            pk[j / 2] = pack_bf16x2(__uint_as_float(v0[j]), __uint_as_float(v0[j + 1]));
-            pk[16 + j / 2] = pack_bf16x2(__uint_as_float(v1[j]), __uint_as_float(v1[j + 1]));
+          for (int c = 0; c < 8; ++c) {
+            const float4 a = *reinterpret_cast<const float4*>(rowp + ((c ^ (lane & 7)) << 4));
+            const float4 b = *reinterpret_cast<const float4*>(rowp + kStageOutBytes + ((c ^ (lane & 7)) << 4));
+            v0[4 * c] = __float_as_uint(__uint_as_float(v0[4 * c]) + a.x);
+            v0[4 * c + 1] = __float_as_uint(__uint_as_float(v0[4 * c + 1]) + a.y);
+            v0[4 * c + 2] = __float_as_uint(__uint_as_float(v0[4 * c + 2]) + a.z);
+            v0[4 * c + 3] = __float_as_uint(__uint_as_float(v0[4 * c + 3]) + a.w);
+            v1[4 * c] = __float_as_uint(__uint_as_float(v1[4 * c]) + b.x);
+            v1[4 * c + 1] = __float_as_uint(__uint_as_float(v1[4 * c + 1]) + b.y);
+            v1[4 * c + 2] = __float_as_uint(__uint_as_float(v1[4 * c + 2]) + b.z);
+            v1[4 * c + 3] = __float_as_uint(__uint_as_float(v1[4 * c + 3]) + b.w);
           }
-          store_slice(pk, col);
+          // this row's 64 bf16 over its own 128 bytes of the first buffer
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* t = c < 4 ? &v0[8 * c] : &v1[8 * (c - 4)];
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(t[0]), __uint_as_float(t[1])),
+                           pack_bf16x2(__uint_as_float(t[2]), __uint_as_float(t[3])),
+                           pack_bf16x2(__uint_as_float(t[4]), __uint_as_float(t[5])),
+                           pack_bf16x2(__uint_as_float(t[6]), __uint_as_float(t[7])));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_out, my_stage, nb * kBN + cs, y);
+            bulk_commit();
+          }
+          ++nstore;
         }
       } else if (!kLogits && (g.epi == kEpiStoreF32 || g.epi == kEpiAddF32)) {
         // 32-column slices: 1 TMEM load -> 32 rows x 128 bytes of fp32

@@ -226,7 +226,10 @@ bool use_pairs() {
 
 template <bool A_MN, bool B_MN>
 gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
-                        const sm100::GemmArgs& g, bool pair, int kind, cudaStream_t stream) {
+                        const sm100::GemmArgs& g, bool pair, int kind, cudaStream_t stream,
+                        const CUtensorMap* taux = nullptr) {
+  // taux: the fp32 accumulator read by kEpiAccToBf16 (any valid map otherwise)
+  const CUtensorMap& tx = taux ? *taux : tout;
   const int tiles = g.tiles_m * g.tiles_n * g.k_splits;
   if (tiles == 0) return GH_OK;
   sm100::GemmArgs ga = g;
@@ -238,14 +241,14 @@ gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
     const int pairs = std::min(tiles, std::max(1, sm_count() / 2));
     ProfileScope prof(kind, stream);
     e = launch_pdl(kern, dim3(2 * pairs), dim3(sm100::kGemmThreads), sm100::GemmCfg<true>::kSmem, stream, 2, ta, tb,
-                   tout, ga);
+                   tout, tx, ga);
   } else {
     auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN, false>;
     if (ensure_smem_limit(kern, sm100::GemmCfg<false>::kSmem) != cudaSuccess) return GH_ERR_CUDA;
     const int grid = std::min(tiles, sm_count());
     ProfileScope prof(kind, stream);
     e = launch_pdl(kern, dim3(grid), dim3(sm100::kGemmThreads), sm100::GemmCfg<false>::kSmem, stream, 1, ta, tb,
-                   tout, ga);
+                   tout, tx, ga);
   }
   note_launch();
   return e == cudaSuccess ? GH_OK : GH_ERR_CUDA;
@@ -535,13 +538,12 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
         // the last chunk adds its product to the fp32 accumulator and rounds
         // the sum to bf16 once, straight into grad_weight
         g4.epi = sm100::kEpiAccToBf16;
-        g4.acc = acc;
-        g4.acc_ld = D;
       }
     } else {
       g4.epi = c == 0 ? sm100::kEpiStoreBf16 : sm100::kEpiBf16Add;
     }
-    st = launch_gemm<true, true>(tm_l_m, tm_x_n, *out4, g4, pair, GH_KERNEL_DW_GEMM, stream);
+    st = launch_gemm<true, true>(tm_l_m, tm_x_n, *out4, g4, pair, GH_KERNEL_DW_GEMM, stream,
+                                 g4.epi == sm100::kEpiAccToBf16 ? &tm_acc : nullptr);
   }
   if (st == GH_OK && !custom) st = ce_reduce_launch(row_loss, N, n_valid, a.mean, a.loss, stream);
   scratch_free(scratch, stream);
