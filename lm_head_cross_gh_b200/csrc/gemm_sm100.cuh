@@ -113,6 +113,11 @@ struct GemmArgs {
   // waits (bounded) until the slice's counter reaches split_target, then sums
   // every k_splits-th row of the slice (counters only grow within a call).
   int split_target;
+  // The chunk's exponentials in the column-blocked layout, through 3-D maps:
+  // a_blocked, the A operand (dX: K-major boxes {64, 128, 1}; dW: M-major boxes
+  // {64, 64, 2}, both 64-column blocks of a CTA's 128 A columns in one copy);
+  // out_blocked, the bf16 output of the epilogue (boxes {64, 32, 1}).
+  int a_blocked, out_blocked;
   // failure-path tests: 1 + the stage of unit 0's first tile whose loads the
   // producer leaves out (0: none)
   int withhold_plus1;
@@ -155,6 +160,32 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       "%4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(map), "r"(bar), "r"(x), "r"(y)
       : "memory");
+}
+
+// 3-D forms for the column-blocked layout of the chunk's exponentials:
+// element (row r, column c) at ((c / 64) * block_rows + r) * 64 + c % 64, so a
+// box of 64 columns and any run of rows is one contiguous piece of memory.
+// Coordinates {c % 64 (always 0 here), r, c / 64}.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                                 int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(map), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
 }
 
 // Allow at most one committed bulk group still reading shared memory.
@@ -466,9 +497,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             tma_load_2d(dst, map, &full[stage], x, y);
           };
+          auto load3 = [&](void* dst, const CUtensorMap* map, int y, int z) {
+            if constexpr (PAIR) {
+              if (!leader) {
+                tma_load_3d_pair(dst, map, map_to_rank(&full[stage], 0), 0, y, z);
+                return;
+              }
+            }
+            tma_load_3d(dst, map, &full[stage], 0, y, z);
+          };
           // the leader's stage barrier counts both CTAs' bytes
           if (leader) mbar_arrive_expect_tx(&full[stage], PAIR ? 2 * kStageBytes : kStageBytes);
-          if constexpr (A_MN) {
+          if (g.a_blocked) {
+            if constexpr (A_MN) load3(sa, &tma_a, k0, m0 >> 6);  // blocks m0/64 and m0/64 + 1
+            else load3(sa, &tma_a, m0, kb);
+          } else if constexpr (A_MN) {
             load(sa, &tma_a, m0, k0);
             load(sa + 8192, &tma_a, m0 + 64, k0);
           } else {
@@ -561,12 +604,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int tile = unit; tile < num_tiles_run; tile += units) {
       int mb, nb, ks;
       tile_coords(tile, mb, nb, ks);
-      if (!wait_or_abort<PAIR>(&tmem_full[acc], acc_phase, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t t_row = tmem_base + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
       const int rbase = mb * C::kTileM + static_cast<int>(rank) * kBM + q * 32;  // this warp's first row
       const int y = ks * g.split_rows + rbase;                                   // its first output row
       const int row = rbase + lane;  // this thread's row of the M rows
+      // the cross-entropy epilogue's per-row inputs, loaded while the tile's MMAs run
+      int64_t row_t = 0;
+      float row_r = 0.0f;
+      if (kLogits && g.epi == kEpiCeExp && row < g.M) {
+        row_t = g.targets[row];
+        if (g.row_ref) row_r = g.row_ref[row];
+      }
+      if (!wait_or_abort<PAIR>(&tmem_full[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
       // 32 rows x 64 bf16 (this warp's slice at column x) to global memory
       // through a 128-byte swizzled staging buffer and one TMA store.
       auto store_slice = [&](const uint32_t (&pk)[32], int x) {
@@ -583,7 +633,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tma_out, buf, x, y);
+          if (g.out_blocked) tma_store_3d(&tma_out, buf, 0, y, x >> 6);
+          else tma_store_2d(&tma_out, buf, x, y);
           bulk_commit();
         }
         ++nstore;
@@ -595,9 +646,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float nr = -INFINITY;
         int tcol = -1;
         if (row < g.M) {
-          const int64_t t = g.targets[row];
+          const int64_t t = row_t;
           if (t != g.ignore_index && t >= 0 && t < g.N) {
-            nr = g.row_ref ? -g.row_ref[row] * kLog2e : 0.0f;
+            nr = -row_r * kLog2e;
             const int64_t off = t - static_cast<int64_t>(nb) * kBN;
             if (off >= 0 && off < kBN) tcol = static_cast<int>(off);
           }
@@ -664,11 +715,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (ce) {
           keep = false;
           if (row < g.M) {
-            const int64_t t = g.targets[row];
+            const int64_t t = row_t;
             keep = t != g.ignore_index && t >= 0 && t < g.N;
             if (keep && t >= static_cast<int64_t>(nb) * kBN && t < static_cast<int64_t>(nb) * kBN + kBN)
               tcol = static_cast<int>(t - static_cast<int64_t>(nb) * kBN);
-            if (g.row_ref) nrl2 = -g.row_ref[row] * kLog2e;
+            nrl2 = -row_r * kLog2e;
           }
         } else if (g.row_scale) {
           rs = row < g.M ? g.row_scale[row] : 0.0f;
@@ -746,7 +797,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tma_out, buf, nb * kBN + cs, y);
+            if (g.out_blocked) tma_store_3d(&tma_out, buf, 0, y, (nb * kBN + cs) >> 6);
+            else tma_store_2d(&tma_out, buf, nb * kBN + cs, y);
             bulk_commit();
           }
           ++nstore;

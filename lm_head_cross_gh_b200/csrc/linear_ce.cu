@@ -81,6 +81,23 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map of a chunk's exponentials P in the column-blocked layout: element
+// (row r, column c) at ((c / 64) * blk_rows + r) * 64 + c % 64, dims {64, rows,
+// nblk}, box {64, box_rows, box_blocks}, 128-byte swizzle.  A box of whole
+// 64-column blocks is contiguous memory, and no box reaches past the array.
+bool make_pblk(CUtensorMap* m, const void* base, uint64_t rows, uint64_t nblk, uint64_t blk_rows, uint32_t box_rows,
+               uint32_t box_blocks) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {64, rows, nblk};
+  const cuuint64_t strides[2] = {128, blk_rows * 128};
+  const cuuint32_t box[3] = {64, box_rows, box_blocks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Output maps of the GEMM epilogue: 32-row boxes of 128 bytes (64 bf16 or 32 fp32).
 bool make_out_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld) {
   return make_tmap(m, base, cols, rows, ld * 2, 32, false, 64);
@@ -107,8 +124,8 @@ struct FinalizeArgs {
   int* flag;                // first pass: set when a row needs the recompute; recompute: runs only if set
   float* alpha;             // [rows]
   float* row_loss;          // [rows] (this chunk's slice)
-  uint16_t* P;              // [rows, ld] exponentials of the chunk
-  int64_t ld;
+  uint16_t* P;              // exponentials of the chunk, column-blocked (blocks of blk_rows x 64)
+  int64_t blk_rows;
   const uint16_t* X;        // [rows, D] inputs of the chunk
   uint16_t* Xs;             // [rows, D] alpha-scaled inputs
 };
@@ -173,7 +190,7 @@ __global__ void __launch_bounds__(kFinWarps * 32) lce_finalize_kernel(FinalizeAr
           alpha = scale * f * expf(R - lse);
           loss = (lse - xt) + a.z * lse * lse;
           // G[t] = alpha (exp(x_t - R) - scale / alpha) = scale ((1 + 2 z lse) p_t - 1)
-          a.P[static_cast<int64_t>(row) * a.ld + t] = to_bf16_bits(expf(xt - R) - scale / alpha);
+          a.P[((t >> 6) * a.blk_rows + row) * 64 + (t & 63)] = to_bf16_bits(expf(xt - R) - scale / alpha);
         }
       }
       a.row_loss[row] = loss;
@@ -351,7 +368,10 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t off_rows = 256;
   const size_t off_buf = up(off_rows + sizeof(float) * N);
-  const size_t buf_bytes = static_cast<size_t>(chunk) * ld * 2;
+  // the chunk buffer: caller-visible row-major logits [chunk, ld] on the
+  // plain path; the exponentials in 64-column blocks on the fused path
+  const int64_t nblk = (V + 63) / 64;
+  const size_t buf_bytes = static_cast<size_t>(chunk) * (fused ? nblk * 64 : ld) * 2;
   const size_t off_acc = up(off_buf + buf_bytes);
   const size_t acc_bytes = acc32 ? static_cast<size_t>(V) * D * 4 : 0;
   const size_t off_ws = up(off_acc + acc_bytes);
@@ -417,9 +437,14 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     // the B operand of dW: the chunk's inputs, scaled by alpha on the fused path
     const uint16_t* Bdw = fused ? Xs : Xc;
     CUtensorMap tm_x_k, tm_l_k, tm_l_m, tm_x_n, tm_l_out, tm_dx_out;
-    if (!make_tmap(&tm_x_k, Xc, D, rows, D * 2, sm100::kBM) || !make_tmap(&tm_l_k, L, V, rows, ld * 2, sm100::kBM) ||
-        !make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) || !make_tmap(&tm_x_n, Bdw, D, rows, D * 2, 64) ||
-        !make_out_bf16(&tm_l_out, L, V, rows, ld) || !make_out_bf16(&tm_dx_out, dX + c0 * D, D, rows, D)) {
+    const bool maps_ok =
+        make_tmap(&tm_x_k, Xc, D, rows, D * 2, sm100::kBM) && make_tmap(&tm_x_n, Bdw, D, rows, D * 2, 64) &&
+        make_out_bf16(&tm_dx_out, dX + c0 * D, D, rows, D) &&
+        (fused ? make_pblk(&tm_l_k, L, rows, nblk, chunk, sm100::kBM, 1) && make_pblk(&tm_l_m, L, rows, nblk, chunk, 64, 2) &&
+                     make_pblk(&tm_l_out, L, rows, nblk, chunk, 32, 1)
+               : make_tmap(&tm_l_k, L, V, rows, ld * 2, sm100::kBM) && make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) &&
+                     make_out_bf16(&tm_l_out, L, V, rows, ld));
+    if (!maps_ok) {
       st = GH_ERR_CUDA;
       break;
     }
@@ -432,6 +457,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       g1.stats = stats;
       g1.stats_ld = static_cast<int>(rows_pad);
       g1.x_target = x_target;
+      g1.out_blocked = 1;
       st = launch_gemm<false, false>(tm_x_k, tm_w_k, tm_l_out, g1, pair, GH_KERNEL_LOGITS_GEMM, stream);
       if (st != GH_OK) break;
       // 2: lse, loss, alpha, the target entries and the scaled inputs
@@ -453,7 +479,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       fa.alpha = alpha;
       fa.row_loss = row_loss + c0;
       fa.P = L;
-      fa.ld = ld;
+      fa.blk_rows = chunk;
       fa.X = Xc;
       fa.Xs = Xs;
       const dim3 fgrid(static_cast<unsigned>((rows + 31) / 32));
@@ -495,6 +521,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     // 3: dX_c = G_c W (K split into fp32 partials when the tiles alone leave SMs idle)
     sm100::GemmArgs g3 = gemm_args(rows, static_cast<int>(D), static_cast<int>(V), 1, sm100::kEpiStoreBf16, pair);
     g3.row_scale = alpha;  // null on the plain path
+    g3.a_blocked = fused;
     const int splits = choose_splits(g3.tiles_m * g3.tiles_n, g3.num_kb, units, sm100::kMaxSplits);
     if (splits > 1 && ws) {
       g3.k_splits = std::min(splits, dx_splits);
@@ -521,6 +548,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
 
     // 4: dW (+)= G_c^T X_c
     sm100::GemmArgs g4 = gemm_args(static_cast<int>(V), static_cast<int>(D), rows, 0, sm100::kEpiStoreBf16, pair);
+    g4.a_blocked = fused;
     // dW reads P and the (scaled) inputs, which the dX GEMM before it waited
     // for before letting dependents launch, and nothing dX writes: its tiles
     // start as dX's CTAs retire; it completes after dX, so the next chunk's
