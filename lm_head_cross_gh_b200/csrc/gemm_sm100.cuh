@@ -116,7 +116,7 @@ struct GemmArgs {
   // The chunk's exponentials in the column-blocked layout, through 3-D maps:
   // a_blocked, the A operand (dX: K-major boxes {64, 128, 1}; dW: M-major boxes
   // {64, 64, 2}, both 64-column blocks of a CTA's 128 A columns in one copy);
-  // out_blocked, the bf16 output of the epilogue (boxes {64, 32, 1}).
+  // out_blocked, the bf16 output of the epilogue (boxes {64, 32, 2}: two column blocks per copy).
   int a_blocked, out_blocked;
   // failure-path tests: 1 + the stage of unit 0's first tile whose loads the
   // producer leaves out (0: none)
@@ -619,23 +619,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t t_row = tmem_base + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
       // 32 rows x 64 bf16 (this warp's slice at column x) to global memory
       // through a 128-byte swizzled staging buffer and one TMA store.
+      // Slices go out in pairs (columns x and x + 64, staged in the warp's two
+      // buffers): one proxy fence and one bulk group per pair, one copy of
+      // both 64-column blocks for the blocked layout (box {64, 32, 2}).
+      // Every tile stages an even number of slices.
       auto store_slice = [&](const uint32_t (&pk)[32], int x) {
-        uint8_t* buf = my_stage + (nstore & 1) * kStageOutBytes;
-        if (nstore >= 2) {
-          if (lane == 0) bulk_wait_read_1();
+        const int b = nstore & 1;
+        if (b == 0 && nstore >= 2) {  // the previous pair's copy has read both buffers
+          if (lane == 0) bulk_wait_read_all();
           __syncwarp();
         }
-        uint8_t* rowp = buf + lane * 128;
+        uint8_t* rowp = my_stage + b * kStageOutBytes + lane * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (g.out_blocked) tma_store_3d(&tma_out, buf, 0, y, x >> 6);
-          else tma_store_2d(&tma_out, buf, x, y);
-          bulk_commit();
+        if (b == 1) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (g.out_blocked) {
+              tma_store_3d(&tma_out, my_stage, 0, y, (x - 64) >> 6);
+            } else {
+              tma_store_2d(&tma_out, my_stage, x - 64, y);
+              tma_store_2d(&tma_out, my_stage + kStageOutBytes, x, y);
+            }
+            bulk_commit();
+          }
         }
         ++nstore;
       };
@@ -778,30 +788,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               v1[j] = __float_as_uint(__uint_as_float(v1[j]) * rs);
             }
           }
-          uint8_t* buf = my_stage + (nstore & 1) * kStageOutBytes;
-          if (nstore >= 2) {
-            if (lane == 0) bulk_wait_read_1();
-            __syncwarp();
-          }
-          uint8_t* rowp = buf + lane * 128;
+          uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t* src = c < 4 ? &v0[c * 8] : &v1[(c - 4) * 8];
-            const uint4 w = make_uint4(
-                pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
-                pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
-                pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
-                pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
-            *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) = w;
+          for (int j = 0; j < 32; j += 2) {
+            pk[j / 2] = pack_bf16x2(__uint_as_float(v0[j]), __uint_as_float(v0[j + 1]));
+            pk[16 + j / 2] = pack_bf16x2(__uint_as_float(v1[j]), __uint_as_float(v1[j + 1]));
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if (g.out_blocked) tma_store_3d(&tma_out, buf, 0, y, (nb * kBN + cs) >> 6);
-            else tma_store_2d(&tma_out, buf, nb * kBN + cs, y);
-            bulk_commit();
-          }
-          ++nstore;
+          store_slice(pk, nb * kBN + cs);
           if (cs + 64 < kBN) tmem_ld_wait(n0, n1);
         }
         if (ce && row < g.M)

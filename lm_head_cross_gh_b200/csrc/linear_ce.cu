@@ -441,7 +441,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
         make_tmap(&tm_x_k, Xc, D, rows, D * 2, sm100::kBM) && make_tmap(&tm_x_n, Bdw, D, rows, D * 2, 64) &&
         make_out_bf16(&tm_dx_out, dX + c0 * D, D, rows, D) &&
         (fused ? make_pblk(&tm_l_k, L, rows, nblk, chunk, sm100::kBM, 1) && make_pblk(&tm_l_m, L, rows, nblk, chunk, 64, 2) &&
-                     make_pblk(&tm_l_out, L, rows, nblk, chunk, 32, 1)
+                     make_pblk(&tm_l_out, L, rows, nblk, chunk, 32, 2)
                : make_tmap(&tm_l_k, L, V, rows, ld * 2, sm100::kBM) && make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) &&
                      make_out_bf16(&tm_l_out, L, V, rows, ld));
     if (!maps_ok) {
