@@ -188,6 +188,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                : "memory");
 }
 
+// tma_store_3d with an L2 eviction policy (createpolicy).
+__device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap* map, const void* smem_src, int x, int y, int z,
+                                                  uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;" ::"l"(
+                   map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z), "l"(policy)
+               : "memory");
+}
+
 // Allow at most one committed bulk group still reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -639,7 +648,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) {
             if (g.out_blocked) {
-              tma_store_3d(&tma_out, my_stage, 0, y, (x - 64) >> 6);
+              // evict first: the chunk's exponentials are larger than L2 and
+              // are read back only by the next kernels, after most of them have
+              // left L2 anyway; the operands that tiles share stay
+              tma_store_3d_hint(&tma_out, my_stage, 0, y, (x - 64) >> 6, l2_policy_evict_first());
             } else {
               tma_store_2d(&tma_out, my_stage, x - 64, y);
               tma_store_2d(&tma_out, my_stage + kStageOutBytes, x, y);
