@@ -178,6 +178,40 @@ gh_status_t gh_linear_ce_shard_f32(const void* inputs, const void* weight, const
 gh_status_t gh_cast_f32_to_bf16(const float* src, void* dst, int64_t n, void* stream);
 
 /*
+ * gh_linear_ce_shard_f32_sliced — gh_linear_ce_shard_f32 whose last weight-
+ * gradient contraction (the last chunk's G^T @ inputs) runs as `dw_slices`
+ * launches over consecutive ranges of weight rows, so that a data-parallel
+ * caller can start the cross-rank sum of the finished rows while the rest are
+ * computed (the weight-gradient reduction overlapped with the chunk loop; the
+ * Greyhound functional API's chunked_linear_cross_entropy with fp32
+ * grad_weight_accum_dtype, sharded by rows).  The pages have no counterpart for
+ * the callback: it is this library's interface for the overlap.
+ *
+ * After enqueuing the launch for weight rows [v0, v1) the call invokes
+ *     on_slice(ctx, v0, v1, stream)
+ * on the calling host thread; rows v0 .. v1-1 of grad_weight_f32 are final
+ * once the work enqueued on `stream` so far has completed (enqueue the
+ * reduction behind it, e.g. an all-reduce ordered after `stream`).  The
+ * ranges come in order, cover [0, V) without overlap and start at multiples of
+ * 256.  on_slice returning anything but GH_OK stops the call, which returns
+ * that status.  With N = 0 the only callback is (0, V), after grad_weight_f32
+ * is zeroed.
+ *   dw_slices  >= 1: the number of ranges (at most one per 256 weight rows).
+ *   max_sms    the sliced launches use at most this many SMs (<= 0: all), so
+ *              that the caller's communication kernels find free SMs.
+ * Results are bit-identical to gh_linear_ce_shard_f32 for any dw_slices and
+ * max_sms (each output tile is computed by one CTA pair in the same order).
+ * Other arguments as for gh_linear_ce_shard_f32.  GH_ERR_INVALID_ARG for
+ * dw_slices < 1 or a null on_slice.
+ */
+typedef gh_status_t (*gh_dw_slice_fn)(void* ctx, int64_t v0, int64_t v1, void* stream);
+gh_status_t gh_linear_ce_shard_f32_sliced(const void* inputs, const void* weight, const int64_t* targets,
+                                          int64_t N, int64_t D, int64_t V, int64_t chunk, int64_t ignore_index,
+                                          gh_reduction_t reduction, float z_mult, const int64_t* n_valid_total,
+                                          float* loss, void* grad_inputs, float* grad_weight_f32, int64_t dw_slices,
+                                          int max_sms, gh_dw_slice_fn on_slice, void* ctx, void* stream);
+
+/*
  * gh_ce_fwd — the cross-entropy loss of gh_ce_fwd_bwd without its gradient:
  * the evaluation form (forward only, nothing kept for a backward), reading the
  * logits once.

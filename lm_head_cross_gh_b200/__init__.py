@@ -49,6 +49,7 @@ _lib = None
 # gh_chunk_loss_fn(ctx, row0, rows, logits, ld, V, loss_accum, stream) -> gh_status_t
 CHUNK_LOSS_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                  ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p)
+DW_SLICE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p)
 
 
 def lib() -> ctypes.CDLL:
@@ -78,6 +79,9 @@ def lib() -> ctypes.CDLL:
     L.gh_linear_ce_shard_f32.argtypes = [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int64,
                                          c_int64, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
     L.gh_linear_ce_shard_f32.restype = c_int
+    L.gh_linear_ce_shard_f32_sliced.argtypes = list(L.gh_linear_ce_shard_f32.argtypes[:-1]) + [
+        c_int64, c_int, DW_SLICE_FN, c_void_p, c_void_p]
+    L.gh_linear_ce_shard_f32_sliced.restype = c_int
     L.gh_cast_f32_to_bf16.argtypes = [c_void_p, c_void_p, c_int64, c_void_p]
     L.gh_cast_f32_to_bf16.restype = c_int
     L.gh_ce_fwd.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int, c_int64, c_int, c_float,
@@ -283,10 +287,17 @@ def gh_linear_ce_shard(inputs, weight, targets, n_valid_total, ignore_index: int
 
 def gh_linear_ce_shard_f32(inputs, weight, targets, n_valid_total, ignore_index: int = -100,
                            reduction: str = "mean", z_loss: float = 0.0, chunk: int = 0, *, grad_inputs=None,
-                           grad_weight_f32=None, loss=None, stream=None):
+                           grad_weight_f32=None, loss=None, stream=None, on_slice=None, dw_slices: int = 1,
+                           max_sms: int = 0):
     """``gh_linear_ce_shard`` with fp32 accumulation whose weight gradient comes
     back as the shard's unrounded fp32 sum (float32 [V, D]), for an fp32
-    cross-rank sum followed by one rounding (``gh_cast_f32_to_bf16``)."""
+    cross-rank sum followed by one rounding (``gh_cast_f32_to_bf16``).
+
+    With ``on_slice`` (``gh_linear_ce_shard_f32_sliced``) the last chunk's
+    weight-gradient launch is cut into ``dw_slices`` ranges of weight rows on
+    at most ``max_sms`` SMs (0: all), and ``on_slice(v0, v1)`` is called, with
+    the library's stream current, after each range is enqueued: rows v0..v1-1
+    of the fp32 gradient are final behind the work enqueued so far."""
     import torch
     _need(inputs.dim() == 2 and weight.dim() == 2 and inputs.shape[1] == weight.shape[1], "shapes")
     _need(inputs.dtype == torch.bfloat16 and weight.dtype == torch.bfloat16, "inputs/weight must be bfloat16")
@@ -306,11 +317,34 @@ def gh_linear_ce_shard_f32(inputs, weight, targets, n_valid_total, ignore_index:
           and grad_weight_f32.is_contiguous(), "grad_weight_f32: contiguous float32 [V, D]")
     if loss is None:
         loss = torch.empty((), dtype=torch.float32, device=inputs.device)
-    st = lib().gh_linear_ce_shard_f32(_ptr(inputs), _ptr(weight), _ptr(targets), N, D, V, int(chunk),
-                                      int(ignore_index), GH_REDUCTION[reduction], float(z_loss),
-                                      _ptr(n_valid_total), _ptr(loss), _ptr(grad_inputs), _ptr(grad_weight_f32),
-                                      _stream_handle(stream))
-    _check(st, "gh_linear_ce_shard_f32")
+    args = (_ptr(inputs), _ptr(weight), _ptr(targets), N, D, V, int(chunk), int(ignore_index),
+            GH_REDUCTION[reduction], float(z_loss), _ptr(n_valid_total), _ptr(loss), _ptr(grad_inputs),
+            _ptr(grad_weight_f32))
+    if on_slice is None:
+        st = lib().gh_linear_ce_shard_f32(*args, _stream_handle(stream))
+        _check(st, "gh_linear_ce_shard_f32")
+        return loss, grad_inputs, grad_weight_f32
+    _need(int(dw_slices) >= 1, "dw_slices >= 1")
+    dev = inputs.device
+    errors = []
+
+    def callback(ctx, v0, v1, stream_ptr):
+        try:
+            strm = (torch.cuda.ExternalStream(stream_ptr, device=dev) if stream_ptr
+                    else torch.cuda.default_stream(dev))
+            with torch.cuda.stream(strm):
+                on_slice(int(v0), int(v1))
+            return GH_OK
+        except BaseException as e:  # reported after the call returns
+            errors.append(e)
+            return GH_ERR_INVALID_ARG
+
+    fn = DW_SLICE_FN(callback)
+    st = lib().gh_linear_ce_shard_f32_sliced(*args, int(dw_slices), int(max_sms), fn, None,
+                                             _stream_handle(stream))
+    if errors:
+        raise errors[0]
+    _check(st, "gh_linear_ce_shard_f32_sliced")
     return loss, grad_inputs, grad_weight_f32
 
 

@@ -237,7 +237,9 @@ gh_status_t gh_selective_log_softmax(const void* logits, const int64_t* index, i
 static gh_status_t linear_ce_impl(const void* inputs, const void* weight, const int64_t* targets, int64_t N,
                                   int64_t D, int64_t V, int64_t chunk, gh_accum_t accum_dtype, int64_t ignore_index,
                                   gh_reduction_t reduction, float z_mult, const int64_t* n_total, float* loss,
-                                  void* grad_inputs, void* grad_weight, void* stream_, float* grad_weight_f32 = nullptr) {
+                                  void* grad_inputs, void* grad_weight, void* stream_, float* grad_weight_f32 = nullptr,
+                                  gh_dw_slice_fn on_slice = nullptr, void* slice_ctx = nullptr,
+                                  int64_t dw_slices = 1, int max_sms = 0) {
   if (N < 0 || D < 1 || V < 1 || V >= (int64_t(1) << 31) || D >= (int64_t(1) << 31)) return GH_ERR_INVALID_ARG;
   if (D % 8) return GH_ERR_INVALID_ARG;
   if (accum_dtype != GH_ACCUM_FP32 && accum_dtype != GH_ACCUM_WEIGHT) return GH_ERR_INVALID_ARG;
@@ -266,6 +268,10 @@ static gh_status_t linear_ce_impl(const void* inputs, const void* weight, const 
   a.dW = grad_weight;
   a.n_total = reinterpret_cast<const unsigned long long*>(n_total);
   a.dW32 = grad_weight_f32;
+  a.on_slice = on_slice;
+  a.slice_ctx = slice_ctx;
+  a.dw_slices = dw_slices;
+  a.max_sms = max_sms;
   return linear_ce_run(a, static_cast<cudaStream_t>(stream_));
 }
 
@@ -295,6 +301,19 @@ gh_status_t gh_linear_ce_shard_f32(const void* inputs, const void* weight, const
   // grad_weight_f32 stands in for the bf16 output in the argument checks
   return linear_ce_impl(inputs, weight, targets, N, D, V, chunk, GH_ACCUM_FP32, ignore_index, reduction, z_mult,
                         n_valid_total, loss, grad_inputs, grad_weight_f32, stream, grad_weight_f32);
+}
+
+gh_status_t gh_linear_ce_shard_f32_sliced(const void* inputs, const void* weight, const int64_t* targets,
+                                          int64_t N, int64_t D, int64_t V, int64_t chunk, int64_t ignore_index,
+                                          gh_reduction_t reduction, float z_mult, const int64_t* n_valid_total,
+                                          float* loss, void* grad_inputs, float* grad_weight_f32, int64_t dw_slices,
+                                          int max_sms, gh_dw_slice_fn on_slice, void* ctx, void* stream) {
+  if (!n_valid_total || (reinterpret_cast<uintptr_t>(n_valid_total) % 8)) return GH_ERR_INVALID_ARG;
+  if (!grad_weight_f32 || (reinterpret_cast<uintptr_t>(grad_weight_f32) % 16)) return GH_ERR_INVALID_ARG;
+  if (dw_slices < 1 || !on_slice) return GH_ERR_INVALID_ARG;
+  return linear_ce_impl(inputs, weight, targets, N, D, V, chunk, GH_ACCUM_FP32, ignore_index, reduction, z_mult,
+                        n_valid_total, loss, grad_inputs, grad_weight_f32, stream, grad_weight_f32, on_slice, ctx,
+                        dw_slices, max_sms);
 }
 
 gh_status_t gh_cast_f32_to_bf16(const float* src, void* dst, int64_t n, void* stream) {

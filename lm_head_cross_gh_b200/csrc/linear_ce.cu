@@ -244,9 +244,11 @@ bool use_pairs() {
 template <bool A_MN, bool B_MN>
 gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
                         const sm100::GemmArgs& g, bool pair, int kind, cudaStream_t stream,
-                        const CUtensorMap* taux = nullptr) {
-  // taux: the fp32 accumulator read by kEpiAccToBf16 (any valid map otherwise)
+                        const CUtensorMap* taux = nullptr, int max_sms = 0) {
+  // taux: the fp32 accumulator read by kEpiAccToBf16 (any valid map otherwise);
+  // max_sms > 0: the launch uses at most that many SMs
   const CUtensorMap& tx = taux ? *taux : tout;
+  const int sms = max_sms > 0 ? std::min(max_sms, sm_count()) : sm_count();
   const int tiles = g.tiles_m * g.tiles_n * g.k_splits;
   if (tiles == 0) return GH_OK;
   sm100::GemmArgs ga = g;
@@ -255,14 +257,14 @@ gh_status_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
   if (pair) {
     auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN, true>;
     if (ensure_smem_limit(kern, sm100::GemmCfg<true>::kSmem) != cudaSuccess) return GH_ERR_CUDA;
-    const int pairs = std::min(tiles, std::max(1, sm_count() / 2));
+    const int pairs = std::min(tiles, std::max(1, sms / 2));
     ProfileScope prof(kind, stream);
     e = launch_pdl(kern, dim3(2 * pairs), dim3(sm100::kGemmThreads), sm100::GemmCfg<true>::kSmem, stream, 2, ta, tb,
                    tout, tx, ga);
   } else {
     auto kern = sm100::gemm_bf16_kernel<A_MN, B_MN, false>;
     if (ensure_smem_limit(kern, sm100::GemmCfg<false>::kSmem) != cudaSuccess) return GH_ERR_CUDA;
-    const int grid = std::min(tiles, sm_count());
+    const int grid = std::min(tiles, std::max(1, sms));
     ProfileScope prof(kind, stream);
     e = launch_pdl(kern, dim3(grid), dim3(sm100::kGemmThreads), sm100::GemmCfg<false>::kSmem, stream, 1, ta, tb,
                    tout, tx, ga);
@@ -335,6 +337,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     if (cudaMemsetAsync(a.loss, 0, sizeof(float), stream) != cudaSuccess) return GH_ERR_CUDA;
     if (a.dW32) {
       if (cudaMemsetAsync(a.dW32, 0, static_cast<size_t>(V) * D * 4, stream) != cudaSuccess) return GH_ERR_CUDA;
+      if (a.on_slice) return a.on_slice(a.slice_ctx, 0, V, stream);
     } else if (cudaMemsetAsync(a.dW, 0, static_cast<size_t>(V) * D * 2, stream) != cudaSuccess) {
       return GH_ERR_CUDA;
     }
@@ -570,8 +573,31 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     } else {
       g4.epi = c == 0 ? sm100::kEpiStoreBf16 : sm100::kEpiBf16Add;
     }
-    st = launch_gemm<true, true>(tm_l_m, tm_x_n, *out4, g4, pair, GH_KERNEL_DW_GEMM, stream,
-                                 g4.epi == sm100::kEpiAccToBf16 ? &tm_acc : nullptr);
+    if (out32 && a.on_slice && c + 1 == nchunks && fused) {
+      // the last contraction in ranges of weight rows (whole tiles), each
+      // handed to the caller once enqueued
+      const int tiles_all = g4.tiles_m;
+      const int slices = static_cast<int>(std::min<int64_t>(std::max<int64_t>(a.dw_slices, 1), tiles_all));
+      for (int s = 0; s < slices && st == GH_OK; ++s) {
+        const int64_t v0 = static_cast<int64_t>(tiles_all) * s / slices * tile_m;
+        const int64_t v1 = std::min<int64_t>(V, static_cast<int64_t>(tiles_all) * (s + 1) / slices * tile_m);
+        CUtensorMap tm_a_s, tm_o_s;
+        if (!make_pblk(&tm_a_s, L + (v0 / 64) * chunk * 64, rows, (v1 - v0 + 63) / 64, chunk, 64, 2) ||
+            !make_out_f32(&tm_o_s, acc + v0 * D, D, v1 - v0, D)) {
+          st = GH_ERR_CUDA;
+          break;
+        }
+        sm100::GemmArgs gs = gemm_args(static_cast<int>(v1 - v0), static_cast<int>(D), rows, 0, g4.epi, pair);
+        gs.a_blocked = 1;
+        gs.defer_wait = 1;
+        st = launch_gemm<true, true>(tm_a_s, tm_x_n, tm_o_s, gs, pair, GH_KERNEL_DW_GEMM, stream, nullptr,
+                                     a.max_sms);
+        if (st == GH_OK) st = a.on_slice(a.slice_ctx, v0, v1, stream);
+      }
+    } else {
+      st = launch_gemm<true, true>(tm_l_m, tm_x_n, *out4, g4, pair, GH_KERNEL_DW_GEMM, stream,
+                                   g4.epi == sm100::kEpiAccToBf16 ? &tm_acc : nullptr);
+    }
   }
   if (st == GH_OK && !custom) st = ce_reduce_launch(row_loss, N, n_valid, a.mean, a.loss, stream);
   scratch_free(scratch, stream);

@@ -26,6 +26,12 @@ struct LinearCeArgs {
   const unsigned long long* n_total;  // non-null: the mean divides by this count (all shards)
   float* dW32;             // non-null (fp32 accumulation only): grad_weight is returned here as the
                            // unrounded fp32 sum over the chunks, [V, D], and dW is not written
+  // dW32 only: the last chunk's weight-gradient launch in dw_slices ranges of
+  // weight rows on at most max_sms SMs, on_slice called after each (null: one launch)
+  gh_dw_slice_fn on_slice;
+  void* slice_ctx;
+  int64_t dw_slices;
+  int max_sms;
 };
 
 // out[i] = bf16(src[i]) (round to nearest even), n elements.

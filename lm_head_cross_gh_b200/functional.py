@@ -190,15 +190,31 @@ def data_parallel_cross_entropy(logits, target, ignore_index: int = -100, reduct
 
 class _DPLinearCE(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, inputs, weight, target, ignore_index, reduction, z, accum, group, ops):
+    def forward(ctx, inputs, weight, target, ignore_index, reduction, z, accum, group, ops, slices, comm_sms):
+        import torch.distributed as dist
         t = target.contiguous()
         n = _all_reduce_sum(ops.gh_count_valid(t, weight.shape[0], ignore_index), group)
         if accum == "fp32":
             # every shard's fp32 accumulator is summed in fp32 and the batch's sum
-            # is rounded to the weight dtype once
-            loss, dX, dW32 = ops.gh_linear_ce_shard_f32(inputs.contiguous(), weight.contiguous(), t, n,
-                                                        ignore_index, reduction, z, 0)
-            dW = ops.gh_cast_f32_to_bf16(_all_reduce_sum(dW32, group))
+            # is rounded to the weight dtype once; the sum of each range of
+            # weight rows starts as soon as the last chunk has computed it, while
+            # the other ranges are still being computed
+            V, D = weight.shape
+            dW32 = torch.empty((V, D), dtype=torch.float32, device=weight.device)
+            works = []
+
+            def on_slice(v0, v1):
+                works.append(dist.all_reduce(dW32[v0:v1], op=dist.ReduceOp.SUM, group=group, async_op=True))
+
+            max_sms = 0
+            if weight.is_cuda and comm_sms > 0:
+                max_sms = max(2, torch.cuda.get_device_properties(weight.device).multi_processor_count - comm_sms)
+            loss, dX, _ = ops.gh_linear_ce_shard_f32(inputs.contiguous(), weight.contiguous(), t, n, ignore_index,
+                                                     reduction, z, 0, grad_weight_f32=dW32, on_slice=on_slice,
+                                                     dw_slices=max(1, int(slices)), max_sms=max_sms)
+            for w in works:
+                w.wait()
+            dW = ops.gh_cast_f32_to_bf16(dW32)
         else:
             # "weight": each shard rounds between its chunks; the shards' sums are
             # added in the weight dtype
@@ -213,15 +229,23 @@ class _DPLinearCE(torch.autograd.Function):
     def backward(ctx, g):
         dX, dW = ctx.saved_tensors
         return (_scaled(dX, g) if ctx.needs_input_grad[0] else None,
-                _scaled(dW, g) if ctx.needs_input_grad[1] else None, None, None, None, None, None, None, None)
+                _scaled(dW, g) if ctx.needs_input_grad[1] else None, None, None, None, None, None, None, None,
+                None, None)
 
 
 def data_parallel_chunked_linear_cross_entropy(inputs, weight, target, ignore_index: int = -100,
                                                reduction: str = "mean", z_loss_multiplier: float = 0.0,
-                                               grad_weight_accum_dtype: str = "fp32", group=None, ops=None):
+                                               grad_weight_accum_dtype: str = "fp32", group=None, ops=None,
+                                               overlap_slices: int = 4, comm_sms: int = 16):
     """``chunked_linear_cross_entropy`` of the whole batch whose rows ``inputs`` /
     ``target`` this rank holds, with the weight replicated: the weight gradient
     is summed over the ranks, in fp32 and rounded once for
-    ``grad_weight_accum_dtype="fp32"``, in the weight dtype for ``"weight"``."""
+    ``grad_weight_accum_dtype="fp32"``, in the weight dtype for ``"weight"``.
+
+    For fp32 accumulation the last chunk's weight-gradient contraction runs in
+    ``overlap_slices`` ranges of weight rows on all but ``comm_sms`` SMs, and
+    each range's all-reduce is issued (asynchronously) as soon as it is
+    enqueued, so the communication of the first ranges overlaps the
+    computation of the rest."""
     return _DPLinearCE.apply(inputs, weight, target, ignore_index, reduction, float(z_loss_multiplier),
-                             grad_weight_accum_dtype, group, _ops(ops))
+                             grad_weight_accum_dtype, group, _ops(ops), int(overlap_slices), int(comm_sms))

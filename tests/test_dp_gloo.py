@@ -50,12 +50,29 @@ class _HostOps:
         loss, G = cls.gh_ce_fwd_bwd_shard(X @ W.T, t, n, ii, reduction, z)
         return loss, G @ W, G.T @ X
 
+    slices_seen = []
+
     @classmethod
-    def gh_linear_ce_shard_f32(cls, X, W, t, n, ii, reduction, z, chunk):
-        """bf16 inputs; the shard's weight gradient as an unrounded fp32 sum."""
+    def gh_linear_ce_shard_f32(cls, X, W, t, n, ii, reduction, z, chunk, *, grad_weight_f32=None,
+                               on_slice=None, dw_slices=1, max_sms=0):
+        """bf16 inputs; the shard's weight gradient as an unrounded fp32 sum.
+        With on_slice: the rows of the gradient handed over in dw_slices
+        consecutive ranges, in order, once each range is written."""
         X64, W64 = X.double(), W.double()
         loss, G = cls.gh_ce_fwd_bwd_shard(X64 @ W64.T, t, n, ii, reduction, z)
-        return loss.float(), (G @ W64).to(X.dtype), (G.T @ X64).float()
+        dW = (G.T @ X64).float()
+        if grad_weight_f32 is None:
+            grad_weight_f32 = dW
+        else:
+            grad_weight_f32.copy_(dW)
+        if on_slice is not None:
+            V = W.shape[0]
+            k = min(dw_slices, V)
+            for s in range(k):
+                v0, v1 = V * s // k, V * (s + 1) // k
+                cls.slices_seen.append((v0, v1))
+                on_slice(v0, v1)
+        return loss.float(), (G @ W64).to(X.dtype), grad_weight_f32
 
     @staticmethod
     def gh_cast_f32_to_bf16(src):
@@ -131,9 +148,10 @@ def _rank_main_fp32(rank, world, port, out):
     Xs = X[rows].to(torch.bfloat16).requires_grad_(True)
     Wr = W.to(torch.bfloat16).requires_grad_(True)
     lin = GF.data_parallel_chunked_linear_cross_entropy(Xs, Wr, t[rows], -100, "mean", 1e-3,
-                                                        grad_weight_accum_dtype="fp32", ops=_HostOps)
+                                                        grad_weight_accum_dtype="fp32", ops=_HostOps,
+                                                        overlap_slices=3)
     lin.backward()
-    out.put((rank, lin.item(), Wr.grad))
+    out.put((rank, lin.item(), Wr.grad, list(_HostOps.slices_seen)))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -160,6 +178,9 @@ def test_two_gloo_ranks_fp32_weight_gradient_is_rounded_once():
     once = (parts[0] + parts[1]).to(torch.bfloat16)
     twice = (parts[0].to(torch.bfloat16) + parts[1].to(torch.bfloat16))
     assert not torch.equal(once, twice)  # the two readings differ on this batch
-    for rank, lin, gw in res:
+    for rank, lin, gw, seen in res:
         assert gw.dtype == torch.bfloat16
+        # every range of weight rows was summed over the ranks (each by its own
+        # asynchronous all-reduce) before the single rounding
+        assert seen == [(0, 11), (11, 22), (22, 33)], rank
         assert torch.equal(gw, once), rank

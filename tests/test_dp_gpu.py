@@ -5,7 +5,9 @@ caller passes; with a total of twice the local count the loss and gradients
 are the oracle's for scale 1 / (2 n_valid).  With the local count they are
 bitwise those of gh_ce_fwd_bwd / gh_linear_ce.  gh_linear_ce_shard_f32 returns
 the weight gradient's unrounded fp32 sum (rounded once by gh_cast_f32_to_bf16
-it is the bf16 entry point's).  The data-parallel functional
+it is the bf16 entry point's); its sliced form (the last weight-gradient
+contraction in ranges of weight rows, a callback after each) is bitwise the
+same.  The data-parallel functional
 wrappers on a one-rank NCCL group (the all-reduces are then identities) give
 the same results as the single-process functions.
 """
@@ -83,6 +85,49 @@ def test_linear_ce_shard_f32_returns_the_unrounded_weight_gradient(cuda_device, 
     ref = r["grad_weight"] / (2 * n_local)   # "sum" scaled by the batch's mean factor
     got = dw32.cpu().numpy().astype(np.float64)
     assert np.linalg.norm(got - ref) <= 1e-2 * np.linalg.norm(ref)
+
+
+@pytest.mark.parametrize("chunk,slices,max_sms", [(256, 3, 0), (0, 1, 0), (256, 1000, 20), (0, 5, 41)])
+def test_linear_ce_shard_f32_sliced_is_bitwise_the_unsliced_call(cuda_device, chunk, slices, max_sms):
+    """The last weight-gradient contraction cut into ranges of weight rows (on
+    fewer SMs) gives bitwise the single launch's results; the callbacks come in
+    order, once per range, cover [0, V) and start at multiples of 256."""
+    q = gh_synth.linear_ce_normal(700, 128, 3001, chunk=chunk, ignore_frac=0.05, w_sigma=0.05, z_loss=1e-4, seed=16)
+    X = torch.from_numpy(q.inputs.view(np.int16)).cuda().view(torch.bfloat16)
+    W = torch.from_numpy(q.weight.view(np.int16)).cuda().view(torch.bfloat16)
+    t = torch.from_numpy(q.targets).cuda()
+    total = torch.tensor(int((q.targets != -100).sum()), dtype=torch.int64, device="cuda")
+    la, dxa, dwa = gh.gh_linear_ce_shard_f32(X, W, t, total, -100, "mean", 1e-4, chunk)
+    ranges = []
+    lb, dxb, dwb = gh.gh_linear_ce_shard_f32(X, W, t, total, -100, "mean", 1e-4, chunk,
+                                             on_slice=lambda v0, v1: ranges.append((v0, v1)),
+                                             dw_slices=slices, max_sms=max_sms)
+    torch.cuda.synchronize()
+    tiles = (3001 + 255) // 256
+    k = min(slices, tiles)
+    assert len(ranges) == k and ranges[0][0] == 0 and ranges[-1][1] == 3001
+    assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+    assert all(v0 % 256 == 0 and v1 > v0 for v0, v1 in ranges)
+    assert la.item() == lb.item() and torch.equal(dxa, dxb)
+    assert torch.equal(dwa.view(torch.int32), dwb.view(torch.int32))
+
+
+def test_linear_ce_shard_f32_sliced_stops_on_a_callback_error(cuda_device):
+    q = gh_synth.linear_ce_normal(300, 64, 1500, chunk=0, seed=17)
+    X = torch.from_numpy(q.inputs.view(np.int16)).cuda().view(torch.bfloat16)
+    W = torch.from_numpy(q.weight.view(np.int16)).cuda().view(torch.bfloat16)
+    t = torch.from_numpy(q.targets).cuda()
+    total = torch.tensor(int((q.targets != -100).sum()), dtype=torch.int64, device="cuda")
+    calls = []
+
+    def fail(v0, v1):
+        calls.append((v0, v1))
+        raise RuntimeError("reduction could not start")
+
+    with pytest.raises(RuntimeError, match="could not start"):
+        gh.gh_linear_ce_shard_f32(X, W, t, total, -100, "mean", 0.0, 0, on_slice=fail, dw_slices=3)
+    torch.cuda.synchronize()
+    assert calls == [(0, 512)]  # the call stopped at the first range
 
 
 def test_cast_f32_to_bf16_rounds_to_nearest_even(cuda_device):
