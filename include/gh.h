@@ -193,10 +193,11 @@ gh_status_t gh_cast_f32_to_bf16(const float* src, void* dst, int64_t n, void* st
  * once the work enqueued on `stream` so far has completed (enqueue the
  * reduction behind it, e.g. an all-reduce ordered after `stream`).  The
  * ranges come in order, cover [0, V) without overlap and start at multiples of
- * 256.  on_slice returning anything but GH_OK stops the call, which returns
+ * 128 (whole output tiles).  on_slice returning anything but GH_OK stops the call, which returns
  * that status.  With N = 0 the only callback is (0, V), after grad_weight_f32
  * is zeroed.
- *   dw_slices  >= 1: the number of ranges (at most one per 256 weight rows).
+ *   dw_slices  >= 1: the number of ranges (at most one per output tile of
+ *              weight rows).
  *   max_sms    the sliced launches use at most this many SMs (<= 0: all), so
  *              that the caller's communication kernels find free SMs.
  * Results are bit-identical to gh_linear_ce_shard_f32 for any dw_slices and

@@ -91,7 +91,8 @@ def test_linear_ce_shard_f32_returns_the_unrounded_weight_gradient(cuda_device, 
 def test_linear_ce_shard_f32_sliced_is_bitwise_the_unsliced_call(cuda_device, chunk, slices, max_sms):
     """The last weight-gradient contraction cut into ranges of weight rows (on
     fewer SMs) gives bitwise the single launch's results; the callbacks come in
-    order, once per range, cover [0, V) and start at multiples of 256."""
+    order, once per range, cover [0, V) and start at multiples of 128 (whole
+    256-row tiles here)."""
     q = gh_synth.linear_ce_normal(700, 128, 3001, chunk=chunk, ignore_frac=0.05, w_sigma=0.05, z_loss=1e-4, seed=16)
     X = torch.from_numpy(q.inputs.view(np.int16)).cuda().view(torch.bfloat16)
     W = torch.from_numpy(q.weight.view(np.int16)).cuda().view(torch.bfloat16)
