@@ -17,14 +17,19 @@
 // in a cluster (cta_group::2: each CTA loads its 128 A rows and 128 of the 256
 // B rows, the leader issues the MMAs, each CTA's TMEM holds its 128 rows).
 // Warp roles in each CTA:
-//   warp 0      TMA producer (one lane): A and B tiles into a ring of
-//               shared-memory stages, 128-byte swizzled; a pair's stage
-//               barrier lives in the leader and counts both CTAs' bytes
+//   warps 0, 6  TMA producers (one lane each, alternate stages): A and B
+//               tiles into a ring of shared-memory stages, 128-byte swizzled;
+//               a pair's stage barrier lives in the leader and counts both
+//               CTAs' bytes.  G_c (the chunk's exponentials) is stored in
+//               64-column blocks and read through 3-D maps, so each A tile of
+//               dX and dW is one contiguous piece of memory
 //   warp 1      TMEM allocator; in the leader, the MMA issuer (one lane):
 //               4 x tcgen05.mma (K=16) per stage, commits release the stage
 //               (in both CTAs) and publish finished accumulators
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
-//               the 32 TMEM lanes its warp id selects), conversion, stores
+//               the 32 TMEM lanes its warp id selects), conversion, and TMA
+//               stores, reduce-adds or read-add-store of the output through
+//               two staging buffers per warp
 // Two accumulators of 256 fp32 columns (all 512 TMEM columns) let the
 // epilogue of one tile overlap the MMAs of the next.  Every wait is bounded
 // (GH_ERR_TIMEOUT, then all roles stop, copies in flight land, the MMAs
