@@ -70,6 +70,8 @@ def test_small_three_ragged_chunks(cuda_device, accum, reduction, z):
 @pytest.mark.parametrize("N,D,V,chunk", [
     (256, 128, 517, 256),     # one chunk, V not a multiple of 8 (padded chunk rows)
     (129, 8, 64, 64),         # minimal D, ragged chunk of one row
+    (50, 16, 17, 32),         # V inside one 64-column block of the exponentials
+    (40, 16, 1, 0),           # one class: zero loss (z = 1e-4 aside) and gradients
     (200, 72, 300, 0),        # D not a multiple of 64, default chunk
     (640, 256, 2049, 384),    # several full N tiles, V just past a tile
     (1000, 768, 5003, 384),   # GPT-2 width, ragged everything
