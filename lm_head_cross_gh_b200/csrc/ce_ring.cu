@@ -418,7 +418,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring_kernel(CeArgs a) {
 // the copies), and the consumers wait for the row's lse once, while the
 // producer's pass-2 copies are already in flight.  Their pass-1 copies mark
 // the lines evict-last and the pass-2 copies evict-first, so the row stays in
-// L2 between the two (the gradient stores are evict-first too).
+// L2 between the two (the gradient stores are evict-first too), and pass 2
+// walks the row backwards: the pieces pass 1 read last are re-read first.
 #ifndef GH_RING_LONG_ROW_BYTES
 #define GH_RING_LONG_ROW_BYTES (120 * 1024)
 #endif
@@ -510,7 +511,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
       auto issue_row = [&](int64_t row, bool first_pass) -> bool {
         const RingRow r = ring_row<ES>(a, row);
         const int np = ring_pieces(r);
-        for (int p = 0; p < np; ++p, ++n) {
+        for (int q = 0; q < np; ++q, ++n) {
+          const int p = (lag0 && !first_pass) ? np - 1 - q : q;  // long rows: pass 2 backwards
           const int s = static_cast<int>(n % kRingSlots);
           if (!wait(&sh.empty[s], ((n / kRingSlots) & 1) ^ 1)) return false;
           if (a.withhold_plus1 != 0 && blockIdx.x == 0 && n + 1 == a.withhold_plus1) continue;  // test of the failure path
@@ -683,8 +685,9 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
     const bool congruent = a.congruent != 0;
     const int64_t tb = lead + t * ES;        // target's byte in the row's chunk space
     const int tc = static_cast<int>(tb >> 4), tj = static_cast<int>((tb & 15) / ES);
-    for (int p = 0; p < np; ++p, ++n) {
+    for (int q = 0; q < np; ++q, ++n) {
       if (static_cast<int>(n % kRingGroups) != grp) continue;
+      const int p = lag0 ? np - 1 - q : q;  // long rows: pass 2 backwards (the producer's order)
       const int s = static_cast<int>(n % kRingSlots);
       if (!__all_sync(0xffffffffu, wait(&sh.full[s], (n / kRingSlots) & 1))) {
         ok = false;
