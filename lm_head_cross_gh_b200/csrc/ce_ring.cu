@@ -137,8 +137,9 @@ __device__ __forceinline__ void raise_ref(MaxSum& st, float cm) {
 
 // 2^y on the FMA pipe for y <= 0 (the MUFU unit is the busiest pipe of the
 // ring; pass 1 sends part of its exponentials here): y is clamped at -125,
-// split into r = round(y) (the 1.5 * 2^23 rounding constant leaves r in the
-// low mantissa bits) and f = y - r in [-0.5, 0.5]; 2^f comes from a degree-5
+// split Cody-Waite style into r = round(y) (the 1.5 * 2^23 rounding constant
+// leaves r in the low mantissa bits) and f = y - r in [-0.5, 0.5]; 2^f comes
+// from a degree-5
 // polynomial (coefficients fitted here to the relative error of 2^f on that
 // interval: 2.3e-7 in fp32 Horner form) and r is added to its exponent field.
 __device__ __forceinline__ float2 exp2_fma2(float2 y) {
