@@ -348,10 +348,20 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   int64_t chunk = a.chunk > 0 ? std::min<int64_t>(a.chunk, N) : default_chunk(N, ld);
   const int64_t nchunks = (N + chunk - 1) / chunk;
   if (chunk > INT32_MAX / 2 || V > INT32_MAX / 2) return GH_ERR_UNSUPPORTED;
-  // fp32 accumulator: library scratch when several chunks must be summed before
-  // the single rounding, or the caller's fp32 output (dW32: no rounding here)
+  const bool custom = a.loss_fn != nullptr;
+  const bool fused = !custom;  // the cross-entropy in the logits GEMM's epilogue
+  // fp32 accumulation on the fused path: the weight gradient of two consecutive
+  // chunks in one contraction (K = both chunks' rows), so the fp32 accumulator
+  // is read and written half as often; the two chunks' exponentials and scaled
+  // inputs sit side by side (chunk 2k in rows [0, chunk), 2k + 1 after it)
+  const int grp = (fused && a.accum == GH_ACCUM_FP32 && nchunks > 1) ? 2 : 1;
+  const int64_t ngroups = (nchunks + grp - 1) / grp;
+  const int64_t blk_rows = grp * chunk;  // rows of one 64-column block of the exponentials
+  // fp32 accumulator: library scratch when several weight-gradient contractions
+  // must be summed before the single rounding, or the caller's fp32 output
+  // (dW32: no rounding here)
   const bool out32 = a.dW32 != nullptr;
-  const bool acc32 = !out32 && a.accum == GH_ACCUM_FP32 && nchunks > 1;
+  const bool acc32 = !out32 && a.accum == GH_ACCUM_FP32 && ngroups > 1;
   const bool pair = use_pairs();
   const int tile_m = pair ? sm100::GemmCfg<true>::kTileM : sm100::GemmCfg<false>::kTileM;
   const int sms = sm_count();
@@ -362,8 +372,6 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const int dx_splits = choose_splits(dx_tiles_max, dx_num_kb, units, sm100::kMaxSplits);
   const int64_t rows_pad = static_cast<int64_t>(tiles_m_max) * tile_m;
 
-  const bool custom = a.loss_fn != nullptr;
-  const bool fused = !custom;  // the cross-entropy in the logits GEMM's epilogue
   const int tiles_n_logits = static_cast<int>((V + sm100::kBN - 1) / sm100::kBN);
 
   // scratch: [counter | row losses | chunk buffer | fp32 dW accumulator | dX split partials |
@@ -374,7 +382,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   // the chunk buffer: caller-visible row-major logits [chunk, ld] on the
   // plain path; the exponentials in 64-column blocks on the fused path
   const int64_t nblk = (V + 63) / 64;
-  const size_t buf_bytes = static_cast<size_t>(chunk) * (fused ? nblk * 64 : ld) * 2;
+  const size_t buf_bytes = static_cast<size_t>(fused ? blk_rows * nblk * 64 : chunk * ld) * 2;
   const size_t off_acc = up(off_buf + buf_bytes);
   const size_t acc_bytes = acc32 ? static_cast<size_t>(V) * D * 4 : 0;
   const size_t off_ws = up(off_acc + acc_bytes);
@@ -386,7 +394,7 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   const size_t off_rmax = up(off_xt + vec_bytes);
   const size_t off_alpha = up(off_rmax + vec_bytes);
   const size_t off_xs = up(off_alpha + vec_bytes);
-  const size_t xs_bytes = fused ? static_cast<size_t>(rows_pad) * D * 2 : 0;
+  const size_t xs_bytes = fused ? static_cast<size_t>((grp - 1) * chunk + rows_pad) * D * 2 : 0;
   const size_t off_flags = up(off_xs + xs_bytes);
   const size_t flags_bytes = fused ? static_cast<size_t>(nchunks) * sizeof(int) : 0;
   const size_t off_count = up(off_flags + flags_bytes);
@@ -436,17 +444,17 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
     const int64_t c0 = c * chunk;
     const int rows = static_cast<int>(std::min<int64_t>(chunk, N - c0));
     const uint16_t* Xc = X + c0 * D;
+    const int m = static_cast<int>(c % grp);     // this chunk's place in its group
+    const int64_t gi = c / grp;                  // the group's index
+    uint16_t* Lm = fused ? L + m * chunk * 64 : L;          // its exponentials (first row)
+    uint16_t* Xsm = fused ? Xs + m * chunk * D : nullptr;  // its scaled inputs
 
-    // the B operand of dW: the chunk's inputs, scaled by alpha on the fused path
-    const uint16_t* Bdw = fused ? Xs : Xc;
-    CUtensorMap tm_x_k, tm_l_k, tm_l_m, tm_x_n, tm_l_out, tm_dx_out;
+    CUtensorMap tm_x_k, tm_l_k, tm_l_out, tm_dx_out;
     const bool maps_ok =
-        make_tmap(&tm_x_k, Xc, D, rows, D * 2, sm100::kBM) && make_tmap(&tm_x_n, Bdw, D, rows, D * 2, 64) &&
-        make_out_bf16(&tm_dx_out, dX + c0 * D, D, rows, D) &&
-        (fused ? make_pblk(&tm_l_k, L, rows, nblk, chunk, sm100::kBM, 1) && make_pblk(&tm_l_m, L, rows, nblk, chunk, 64, 2) &&
-                     make_pblk(&tm_l_out, L, rows, nblk, chunk, 32, 2)
-               : make_tmap(&tm_l_k, L, V, rows, ld * 2, sm100::kBM) && make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) &&
-                     make_out_bf16(&tm_l_out, L, V, rows, ld));
+        make_tmap(&tm_x_k, Xc, D, rows, D * 2, sm100::kBM) && make_out_bf16(&tm_dx_out, dX + c0 * D, D, rows, D) &&
+        (fused ? make_pblk(&tm_l_k, Lm, rows, nblk, blk_rows, sm100::kBM, 1) &&
+                     make_pblk(&tm_l_out, Lm, rows, nblk, blk_rows, 32, 2)
+               : make_tmap(&tm_l_k, L, V, rows, ld * 2, sm100::kBM) && make_out_bf16(&tm_l_out, L, V, rows, ld));
     if (!maps_ok) {
       st = GH_ERR_CUDA;
       break;
@@ -481,10 +489,10 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       fa.flag = flags + c;
       fa.alpha = alpha;
       fa.row_loss = row_loss + c0;
-      fa.P = L;
-      fa.blk_rows = chunk;
+      fa.P = Lm;
+      fa.blk_rows = blk_rows;
       fa.X = Xc;
-      fa.Xs = Xs;
+      fa.Xs = Xsm;
       const dim3 fgrid(static_cast<unsigned>((rows + 31) / 32));
       {
         ProfileScope prof(GH_KERNEL_CHUNK_CE, stream);
@@ -549,24 +557,34 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
       if (st != GH_OK) break;
     }
 
-    // 4: dW (+)= G_c^T X_c
-    sm100::GemmArgs g4 = gemm_args(static_cast<int>(V), static_cast<int>(D), rows, 0, sm100::kEpiStoreBf16, pair);
+    // 4: dW (+)= G^T X over the group's chunks, once its last chunk is done
+    if (m + 1 < grp && c + 1 < nchunks) continue;
+    const int64_t g0 = gi * grp * chunk;                                   // the group's first row
+    const int grows = static_cast<int>(std::min<int64_t>(grp * chunk, N - g0));  // its rows (K)
+    // the B operand of dW: the inputs, scaled by alpha on the fused path
+    CUtensorMap tm_l_m, tm_x_n;
+    if (!(fused ? make_pblk(&tm_l_m, L, grows, nblk, blk_rows, 64, 2) && make_tmap(&tm_x_n, Xs, D, grows, D * 2, 64)
+                : make_tmap(&tm_l_m, L, V, rows, ld * 2, 64) && make_tmap(&tm_x_n, Xc, D, rows, D * 2, 64))) {
+      st = GH_ERR_CUDA;
+      break;
+    }
+    sm100::GemmArgs g4 = gemm_args(static_cast<int>(V), static_cast<int>(D), grows, 0, sm100::kEpiStoreBf16, pair);
     g4.a_blocked = fused;
     // dW reads P and the (scaled) inputs, which the dX GEMM before it waited
     // for before letting dependents launch, and nothing dX writes: its tiles
     // start as dX's CTAs retire; it completes after dX, so the next chunk's
-    // logits GEMM cannot overwrite P while dX reads it.
+    // logits GEMM cannot overwrite P while dW reads it.
     g4.defer_wait = 1;
     const CUtensorMap* out4 = &tm_dw_out;
     if (out32) {
-      g4.epi = c == 0 ? sm100::kEpiStoreF32 : sm100::kEpiAddF32;
+      g4.epi = gi == 0 ? sm100::kEpiStoreF32 : sm100::kEpiAddF32;
       out4 = &tm_acc;
     } else if (a.accum == GH_ACCUM_FP32) {
-      if (acc32 && c + 1 < nchunks) {
-        g4.epi = c == 0 ? sm100::kEpiStoreF32 : sm100::kEpiAddF32;
+      if (acc32 && gi + 1 < ngroups) {
+        g4.epi = gi == 0 ? sm100::kEpiStoreF32 : sm100::kEpiAddF32;
         out4 = &tm_acc;
       } else if (acc32) {
-        // the last chunk adds its product to the fp32 accumulator and rounds
+        // the last group adds its product to the fp32 accumulator and rounds
         // the sum to bf16 once, straight into grad_weight
         g4.epi = sm100::kEpiAccToBf16;
       }
@@ -582,12 +600,12 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
         const int64_t v0 = static_cast<int64_t>(tiles_all) * s / slices * tile_m;
         const int64_t v1 = std::min<int64_t>(V, static_cast<int64_t>(tiles_all) * (s + 1) / slices * tile_m);
         CUtensorMap tm_a_s, tm_o_s;
-        if (!make_pblk(&tm_a_s, L + (v0 / 64) * chunk * 64, rows, (v1 - v0 + 63) / 64, chunk, 64, 2) ||
+        if (!make_pblk(&tm_a_s, L + (v0 / 64) * blk_rows * 64, grows, (v1 - v0 + 63) / 64, blk_rows, 64, 2) ||
             !make_out_f32(&tm_o_s, acc + v0 * D, D, v1 - v0, D)) {
           st = GH_ERR_CUDA;
           break;
         }
-        sm100::GemmArgs gs = gemm_args(static_cast<int>(v1 - v0), static_cast<int>(D), rows, 0, g4.epi, pair);
+        sm100::GemmArgs gs = gemm_args(static_cast<int>(v1 - v0), static_cast<int>(D), grows, 0, g4.epi, pair);
         gs.a_blocked = 1;
         gs.defer_wait = 1;
         st = launch_gemm<true, true>(tm_a_s, tm_x_n, tm_o_s, gs, pair, GH_KERNEL_DW_GEMM, stream, nullptr,
