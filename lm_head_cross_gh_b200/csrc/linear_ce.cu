@@ -353,8 +353,13 @@ gh_status_t linear_ce_run(const LinearCeArgs& a, cudaStream_t stream) {
   // fp32 accumulation on the fused path: the weight gradient of two consecutive
   // chunks in one contraction (K = both chunks' rows), so the fp32 accumulator
   // is read and written half as often; the two chunks' exponentials and scaled
-  // inputs sit side by side (chunk 2k in rows [0, chunk), 2k + 1 after it)
-  const int grp = (fused && a.accum == GH_ACCUM_FP32 && nchunks > 1) ? 2 : 1;
+  // inputs sit side by side (chunk 2k in rows [0, chunk), 2k + 1 after it).
+  // Only while the pair's scaled inputs (the B operand every tile of the
+  // contraction reads) stay well inside L2: at 67 MB (the Llama-3-8B head) the
+  // pair contraction re-read them from DRAM and the step's DRAM traffic grew
+  // by a third.
+  constexpr int64_t kPairDwMaxBytes = int64_t(32) << 20;
+  const int grp = (fused && a.accum == GH_ACCUM_FP32 && nchunks > 1 && 2 * chunk * D * 2 <= kPairDwMaxBytes) ? 2 : 1;
   const int64_t ngroups = (nchunks + grp - 1) / grp;
   const int64_t blk_rows = grp * chunk;  // rows of one 64-column block of the exponentials
   // fp32 accumulator: library scratch when several weight-gradient contractions
