@@ -281,8 +281,13 @@ gh_status_t gh_selective_log_softmax(const void* logits, const int64_t* index, i
  *   grad_inputs  [N, D] bf16, device, written.
  *   grad_weight  [V, D] bf16, device, written (overwritten, not added to).
  *   stream       cudaStream_t as void*.
- * Scratch (stream-ordered): chunk x round_up(V, 8) bf16 logits/gradient,
- * an fp32 [V, D] accumulator when accum_dtype == GH_ACCUM_FP32, and O(N) floats.
+ * Scratch (stream-ordered): the chunk's exponentials, chunk x round_up(V, 64)
+ * bf16 (twice that with fp32 accumulation over several chunks when
+ * 2 x chunk x D x 2 bytes <= 32 MiB: two chunks then share one weight-gradient
+ * contraction), an fp32 [V, D] accumulator when fp32 accumulation needs more
+ * than one contraction, the chunk's scaled inputs (chunk or 2 x chunk rows
+ * x D bf16), per-tile row statistics (ceil(V / 256) x chunk float2) and O(N)
+ * floats.
  */
 gh_status_t gh_linear_ce(const void* inputs, const void* weight, const int64_t* targets,
                          int64_t N, int64_t D, int64_t V, int64_t chunk, gh_accum_t accum_dtype,
