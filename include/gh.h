@@ -102,6 +102,8 @@ typedef enum { GH_F32 = 0, GH_BF16 = 1 } gh_dtype_t;
  *            as the raw kernel helper on the Greyhound page does); any other
  *            overlap is not.
  *   stream   cudaStream_t as void*.
+ * Non-finite logits follow the definition: a NaN in a valid row makes the loss
+ * NaN and every gradient element of that row NaN; ignored rows are not read.
  */
 gh_status_t gh_ce_fwd_bwd(const void* logits, const int64_t* targets, int64_t B, int64_t V,
                           gh_dtype_t dtype, int64_t ignore_index, gh_reduction_t reduction,
@@ -386,6 +388,23 @@ typedef enum {
   GH_DEBUG_WITHHOLD_GEMM_STAGE = 2
 } gh_debug_t;
 gh_status_t gh_debug_set(gh_debug_t knob, int64_t value);
+
+/*
+ * gh_exp2_eval — out[i] = 2^y[i] for i < n by one of the two routes the
+ * cross-entropy kernels use for their exponentials, so each can be checked on
+ * its own (diagnostic; the Greyhound API has no counterpart):
+ *   method 0  ex2.approx.ftz.f32 on the MUFU pipe (every kernel; results below
+ *             2^-126 flush to zero);
+ *   method 1  the FMA-pipe form of the two-pass ring's long rows: y clamped at
+ *             -125, split into r = round(y) and f = y - r in [-0.5, 0.5], 2^f
+ *             from a degree-5 polynomial fitted to its relative error on that
+ *             interval, r added to the exponent field.  Defined for y <= 0 (the
+ *             kernels' arguments are differences from a running maximum).
+ * y and out: n float32 values, device, caller-owned; may be the same buffer.
+ * Asynchronous on `stream`.  GH_ERR_INVALID_ARG for n < 0, an unknown method
+ * or a NULL pointer with n > 0; GH_ERR_CUDA if the launch fails.
+ */
+gh_status_t gh_exp2_eval(const float* y, float* out, int64_t n, int method, void* stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char* gh_status_string(gh_status_t status);

@@ -112,6 +112,8 @@ def lib() -> ctypes.CDLL:
     L.gh_launch_count.restype = c_int64
     L.gh_debug_set.argtypes = [c_int, c_int64]
     L.gh_debug_set.restype = c_int
+    L.gh_exp2_eval.argtypes = [c_void_p, c_void_p, c_int64, c_int, c_void_p]
+    L.gh_exp2_eval.restype = c_int
     _lib = L
     return L
 
@@ -562,6 +564,19 @@ def gh_debug_set(knob: str, value: int) -> None:
     _check(lib().gh_debug_set(GH_DEBUG[knob], int(value)), "gh_debug_set")
 
 
+def gh_exp2_eval(y, method: str, out=None, stream=None):
+    """2^y of a float32 CUDA tensor by one of the kernels' two routes:
+    ``"mufu"`` (ex2.approx) or ``"fma"`` (the FMA-pipe polynomial, y <= 0)."""
+    import torch
+    _need(y.dtype == torch.float32 and y.is_cuda and y.is_contiguous(), "y: contiguous CUDA float32")
+    if out is None:
+        out = torch.empty_like(y)
+    _need(out.dtype == torch.float32 and out.numel() == y.numel() and out.is_contiguous(), "out")
+    m = {"mufu": 0, "fma": 1}[method]
+    _check(lib().gh_exp2_eval(_ptr(y), _ptr(out), y.numel(), m, _stream_handle(stream)), "gh_exp2_eval")
+    return out
+
+
 def gh_profile_read(kind: str):
     """(summed milliseconds, launches) recorded for one kernel kind."""
     ms = ctypes.c_double(0.0)
@@ -585,7 +600,7 @@ __all__ = [
     "gh_ce_fwd_bwd", "gh_ce_fwd_bwd_noalloc", "GH_NOALLOC_MAX_ROWS", "gh_ce_fwd", "gh_selective_log_softmax",
     "gh_ce_vjp", "gh_linear_ce", "gh_chunked_linear_loss", "CHUNK_LOSS_FN",
     "gh_count_valid", "gh_ce_fwd_bwd_shard", "gh_linear_ce_shard", "gh_linear_ce_shard_f32",
-    "gh_cast_f32_to_bf16",
+    "gh_cast_f32_to_bf16", "gh_exp2_eval",
     "gh_get_device_status", "gh_profile_enable", "gh_profile_read", "gh_debug_set", "GH_DEBUG",
     "gh_launch_count", "GH_KERNEL",
     "GH_OK", "GH_ERR_INVALID_ARG", "GH_ERR_UNSUPPORTED", "GH_ERR_ALLOC", "GH_ERR_CUDA",

@@ -323,6 +323,13 @@ gh_status_t gh_cast_f32_to_bf16(const float* src, void* dst, int64_t n, void* st
   return cast_f32_bf16_launch(src, dst, n, static_cast<cudaStream_t>(stream));
 }
 
+gh_status_t gh_exp2_eval(const float* y, float* out, int64_t n, int method, void* stream) {
+  if (n < 0 || (method != 0 && method != 1)) return GH_ERR_INVALID_ARG;
+  if (n > 0 && (!y || !out)) return GH_ERR_INVALID_ARG;
+  if (n > (int64_t(1) << 40)) return GH_ERR_UNSUPPORTED;
+  return exp2_eval_launch(y, out, n, method, static_cast<cudaStream_t>(stream));
+}
+
 gh_status_t gh_chunked_linear_loss(const void* inputs, const void* weight, int64_t N, int64_t D, int64_t V,
                                    int64_t chunk, gh_accum_t accum_dtype, gh_chunk_loss_fn loss_fn, void* ctx,
                                    float* loss, void* grad_inputs, void* grad_weight, void* stream_) {

@@ -54,6 +54,8 @@ gh_status_t ce_launch(const CeArgs& args, int64_t B, gh_dtype_t dtype, cudaStrea
 // kModeFwdBwd twice (the second copy from L2) and store the gradient.
 int ce_ring_smem_bytes();
 gh_status_t ce_ring_launch(const CeArgs& args, int elem_bytes, int grid, cudaStream_t stream);
+// 2^y[i] -> out[i] by ex2.approx (method 0) or the ring's FMA-pipe polynomial (method 1).
+gh_status_t exp2_eval_launch(const float* y, float* out, int64_t n, int method, cudaStream_t stream);
 // Per-row cross-entropy VJP (ce_vjp.cu).
 gh_status_t ce_vjp_launch(const void* logits, const int64_t* targets, const float* row_loss, const float* g,
                           void* grad, int64_t B, int64_t V, int64_t ignore_index, gh_dtype_t dtype,

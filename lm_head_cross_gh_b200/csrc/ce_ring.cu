@@ -136,15 +136,23 @@ __device__ __forceinline__ void raise_ref(MaxSum& st, float cm) {
 }
 
 // 2^y on the FMA pipe for y <= 0 (the MUFU unit is the busiest pipe of the
-// ring; pass 1 sends part of its exponentials here): y is clamped at -125,
-// split Cody-Waite style into r = round(y) (the 1.5 * 2^23 rounding constant
-// leaves r in the low mantissa bits) and f = y - r in [-0.5, 0.5]; 2^f comes
-// from a degree-5
-// polynomial (coefficients fitted here to the relative error of 2^f on that
-// interval: 2.3e-7 in fp32 Horner form) and r is added to its exponent field.
+// ring; pass 1 sends part of its exponentials here): y is clamped at -125
+// (max.NaN: a NaN stays NaN), split Cody-Waite style into r = round(y) (the
+// 1.5 * 2^23 rounding constant leaves r in the low mantissa bits) and
+// f = y - r in [-0.5, 0.5]; 2^f comes from a degree-5 polynomial
+// (coefficients fitted here to the relative error of 2^f on that interval:
+// 2.3e-7 in fp32 Horner form), multiplied by 2^r built in the exponent field
+// (exact: r >= -125 keeps both factors and the product normal, and a NaN
+// argument makes a NaN product, as ex2.approx does).
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 __device__ __forceinline__ float2 exp2_fma2(float2 y) {
-  y.x = fmaxf(y.x, -125.0f);
-  y.y = fmaxf(y.y, -125.0f);
+  y.x = max_nan(y.x, -125.0f);
+  y.y = max_nan(y.y, -125.0f);
   const float2 t = __fadd2_rn(y, make_float2(12582912.0f, 12582912.0f));
   const float2 r = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
   const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), y);
@@ -154,8 +162,10 @@ __device__ __forceinline__ float2 exp2_fma2(float2 y) {
   p = __ffma2_rn(p, f, make_float2(0.24022120237350464f, 0.24022120237350464f));
   p = __ffma2_rn(p, f, make_float2(0.6931469440460205f, 0.6931469440460205f));
   p = __ffma2_rn(p, f, make_float2(1.0000001192092896f, 1.0000001192092896f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+  // 2^r: r << 23 (the low bits of t shifted into the exponent field) + the bias
+  const float2 s2 = make_float2(__int_as_float((__float_as_int(t.x) << 23) + (127 << 23)),
+                                __int_as_float((__float_as_int(t.y) << 23) + (127 << 23)));
+  return __fmul2_rn(p, s2);
 }
 
 // Of a thread's 8 chunks of a piece, this many take their pass-1 exponentials
@@ -808,6 +818,17 @@ __global__ void __launch_bounds__(kRingThreads, 1) ce_ring2_kernel(CeArgs a) {
   }
 }
 
+// 2^y for n values, by either route the kernels take: method 0 ex2.approx (the
+// MUFU pipe), method 1 exp2_fma2 (the FMA pipe, y <= 0).  Diagnostic only.
+__global__ void exp2_eval_kernel(const float* __restrict__ y, float* __restrict__ out, int64_t n, int method) {
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float y0 = y[i], y1 = i + 1 < n ? y[i + 1] : 0.0f;
+  const float2 r = method == 1 ? exp2_fma2(make_float2(y0, y1)) : make_float2(ex2(y0), ex2(y1));
+  out[i] = r.x;
+  if (i + 1 < n) out[i + 1] = r.y;
+}
+
 using RingKernel = void (*)(CeArgs);
 
 template <typename T>
@@ -822,6 +843,15 @@ RingKernel ring_kernel_for(int es, int mode) {
 }  // namespace
 
 int ce_ring_smem_bytes() { return kRingHdrBytes + kRingSlots * kRingPieceBytes; }
+
+gh_status_t exp2_eval_launch(const float* y, float* out, int64_t n, int method, cudaStream_t stream) {
+  if (n == 0) return GH_OK;
+  constexpr int kThreads = 256;
+  const int64_t blocks = ((n + 1) / 2 + kThreads - 1) / kThreads;
+  note_launch();
+  exp2_eval_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(y, out, n, method);
+  return cudaGetLastError() == cudaSuccess ? GH_OK : GH_ERR_CUDA;
+}
 
 gh_status_t ce_ring_launch(const CeArgs& args, int es, int grid, cudaStream_t stream) {
   CeArgs a = args;

@@ -145,6 +145,32 @@ def test_empty_batch_writes_zero_loss(cuda_device):
     assert loss.item() == 0.0
 
 
+@pytest.mark.parametrize("V", [50257, 65543])
+def test_nan_logit_poisons_its_row_only(cuda_device, V):
+    """A NaN logit in a valid row makes the loss NaN and that row's gradient
+    NaN (as the definition's sum over the row does), whichever part of the
+    row holds it: on the ring's long rows (65543 bf16 columns, 128 KiB) column
+    1000 is evaluated on the FMA-pipe exponential and column 20000 on the MUFU
+    one.  Other rows stay finite, and a NaN in an ignored row is not read."""
+    p = gh_synth.ce_normal(6, V, 3.0, dtype="bf16", reduction="sum", seed=7)
+    x, t = to_device(p)
+    t[4] = -100
+    x[4, 9] = float("nan")
+    loss, grad = gh.gh_ce_fwd_bwd(x, t, -100, "sum", 0.0)
+    assert torch.isfinite(loss).item() and torch.isfinite(grad).all().item()
+    assert not grad[4].any().item()
+    for col in (1000, 20000):
+        y = x.clone()
+        y[2, col] = float("nan")
+        loss, grad = gh.gh_ce_fwd_bwd(y, t, -100, "sum", 0.0)
+        torch.cuda.synchronize()
+        assert torch.isnan(loss).item(), col
+        assert torch.isnan(grad[2].float()).all().item(), col
+        keep = [0, 1, 3, 5]
+        assert torch.isfinite(grad[keep].float()).all().item(), col
+        assert not grad[4].any().item()
+
+
 def test_results_are_deterministic(cuda_device):
     p = gh_synth.ce_normal(64, 50257, 3.0, dtype="bf16", ignore_frac=0.02, z_loss=1e-4, seed=11)
     x, t = to_device(p)
