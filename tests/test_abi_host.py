@@ -110,3 +110,25 @@ def test_newer_entry_points_reject_bad_arguments_on_host(L):
     # gh_chunked_linear_loss needs a callback
     assert L.gh_chunked_linear_loss(lg, FAKE + (4 << 32), 64, 64, 100, 0, 0, gh.CHUNK_LOSS_FN(), None, out,
                                     FAKE + (5 << 32), FAKE + (6 << 32), None) == bad
+
+
+def test_plain_c_program_uses_the_header_and_library(L, tmp_path):
+    """include/gh.h compiles as C99 with warnings as errors, and a C program
+    linked against libgh.so gets every host-side refusal the header promises
+    (tests/abi_c_check.c), with no GPU and no Python in between."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(gh.LIB_PATH)
+    exe = str(tmp_path / "abi_c_check")
+    build = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                            "-I", os.path.join(root, "include"), os.path.join(root, "tests", "abi_c_check.c"),
+                            "-o", exe, "-L", libdir, "-lgh", "-Wl,-rpath," + libdir, "-lm"],
+                           capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert "0 failed checks" in run.stdout
