@@ -67,7 +67,7 @@ extern "C" {
 typedef enum {
   GH_OK = 0,
   GH_ERR_INVALID_ARG = 1,  /* rejected on the host; nothing was enqueued */
-  GH_ERR_UNSUPPORTED = 2,  /* valid request outside what this build supports */
+  GH_ERR_UNSUPPORTED = 2,  /* valid request outside what this library version supports */
   GH_ERR_ALLOC = 3,        /* scratch allocation failed; nothing was enqueued */
   GH_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed */
   GH_ERR_TIMEOUT = 5,      /* a bounded device wait ran out (device status) */
