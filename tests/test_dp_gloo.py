@@ -89,6 +89,13 @@ def _batch(seed=0, N=24, D=6, V=17):
     return X, W, t
 
 
+def _plain(t):
+    """A tensor as a numpy copy for the result queue: a torch tensor put on a
+    multiprocessing queue travels as a shared file descriptor, which the
+    parent can no longer fetch once the rank has exited."""
+    return t.detach().float().numpy().copy() if t.dtype == torch.bfloat16 else t.detach().numpy().copy()
+
+
 def _rank_main(rank, world, port, out):
     os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import torch.distributed as dist
@@ -106,7 +113,7 @@ def _rank_main(rank, world, port, out):
     lin = GF.data_parallel_chunked_linear_cross_entropy(Xs, Wr, t[rows], -100, "mean", 1e-3,
                                                         grad_weight_accum_dtype="weight", ops=_HostOps)
     lin.backward()
-    out.put((rank, loss.item(), logits.grad, lin.item(), Xs.grad, Wr.grad))
+    out.put((rank, loss.item(), _plain(logits.grad), lin.item(), _plain(Xs.grad), _plain(Wr.grad)))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -128,6 +135,7 @@ def test_two_gloo_ranks_data_parallel_cross_entropy():
     n = int((t != -100).sum())
     lf, Gf = _HostOps.gh_ce_fwd_bwd_shard(X @ W.T, t, n, -100, "mean", 1e-3)
     for rank, loss, glog, lin, gx, gw in res:
+        glog, gx, gw = torch.from_numpy(glog), torch.from_numpy(gx), torch.from_numpy(gw)
         rows = slice(rank * 12, (rank + 1) * 12)
         assert loss == pytest.approx(lf.item(), rel=1e-12)
         assert torch.allclose(glog, Gf[rows], rtol=1e-12, atol=1e-15)
@@ -151,7 +159,7 @@ def _rank_main_fp32(rank, world, port, out):
                                                         grad_weight_accum_dtype="fp32", ops=_HostOps,
                                                         overlap_slices=3)
     lin.backward()
-    out.put((rank, lin.item(), Wr.grad, list(_HostOps.slices_seen)))
+    out.put((rank, lin.item(), str(Wr.grad.dtype), _plain(Wr.grad), list(_HostOps.slices_seen)))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -178,8 +186,9 @@ def test_two_gloo_ranks_fp32_weight_gradient_is_rounded_once():
     once = (parts[0] + parts[1]).to(torch.bfloat16)
     twice = (parts[0].to(torch.bfloat16) + parts[1].to(torch.bfloat16))
     assert not torch.equal(once, twice)  # the two readings differ on this batch
-    for rank, lin, gw, seen in res:
-        assert gw.dtype == torch.bfloat16
+    for rank, lin, gw_dtype, gw, seen in res:
+        assert gw_dtype == str(torch.bfloat16)
+        gw = torch.from_numpy(gw).to(torch.bfloat16)  # bf16 -> fp32 -> bf16 is exact
         # every range of weight rows was summed over the ranks (each by its own
         # asynchronous all-reduce) before the single rounding
         assert seen == [(0, 11), (11, 22), (22, 33)], rank
