@@ -402,7 +402,8 @@ gh_status_t gh_debug_set(gh_debug_t knob, int64_t value);
  *             kernels' arguments are differences from a running maximum).
  * y and out: n float32 values, device, caller-owned; may be the same buffer.
  * Asynchronous on `stream`.  GH_ERR_INVALID_ARG for n < 0, an unknown method
- * or a NULL pointer with n > 0; GH_ERR_CUDA if the launch fails.
+ * or a NULL pointer with n > 0; GH_ERR_UNSUPPORTED for n > 2^32; GH_ERR_CUDA
+ * if the launch fails.
  */
 gh_status_t gh_exp2_eval(const float* y, float* out, int64_t n, int method, void* stream);
 

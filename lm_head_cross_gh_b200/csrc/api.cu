@@ -326,7 +326,7 @@ gh_status_t gh_cast_f32_to_bf16(const float* src, void* dst, int64_t n, void* st
 gh_status_t gh_exp2_eval(const float* y, float* out, int64_t n, int method, void* stream) {
   if (n < 0 || (method != 0 && method != 1)) return GH_ERR_INVALID_ARG;
   if (n > 0 && (!y || !out)) return GH_ERR_INVALID_ARG;
-  if (n > (int64_t(1) << 40)) return GH_ERR_UNSUPPORTED;
+  if (n > (int64_t(1) << 32)) return GH_ERR_UNSUPPORTED;  // keeps the grid far inside gridDim.x's limit
   return exp2_eval_launch(y, out, n, method, static_cast<cudaStream_t>(stream));
 }
 

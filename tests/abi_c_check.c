@@ -84,6 +84,7 @@ int main(void) {
   BAD(gh_exp2_eval((const float*)addr(5), (float*)addr(6), -1, 0, NULL));
   BAD(gh_exp2_eval((const float*)addr(5), (float*)addr(6), 4, 2, NULL));
   BAD(gh_exp2_eval(NULL, NULL, 4, 1, NULL));
+  EXPECT(gh_exp2_eval((const float*)addr(5), (float*)addr(6), ((int64_t)1 << 32) + 1, 0, NULL) == GH_ERR_UNSUPPORTED);
   BAD(gh_profile_read((gh_kernel_t)GH_KERNEL_KINDS, NULL, NULL));
   BAD(gh_debug_set((gh_debug_t)9, 0));
   EXPECT(gh_debug_set(GH_DEBUG_WITHHOLD_RING_PIECE, -1) == GH_OK);
