@@ -70,3 +70,75 @@ def test_traffic_entries_are_backed_by_a_summary_and_read_back():
         assert bench.profiled_traffic(e["kernel"], e["source_sha"], e["workload"]) == \
             float(e["traffic_bytes_per_launch"])
         assert bench.profiled_traffic(e["kernel"], "0" * 12, e["workload"]) is None
+
+
+# --------------------------------------------------------------------------
+# the roofline arithmetic bench.py reports (no GPU: fake timings)
+# --------------------------------------------------------------------------
+
+def test_linear_roofline_is_the_whole_step_over_the_burst_peak():
+    """frac = 6 N V D per step / step time / the dense bf16 peak (burst for a
+    timed region under two seconds, sustained beyond, and labelled so); each
+    GEMM's own rate is its third of the step's FLOPs over its launches; the
+    step's DRAM traffic is the profiled bytes of each GEMM launch times its
+    launches per step."""
+    import types
+    import bench
+    N, V, D, steps = 8192, 50257, 768, 20
+    flops = 6.0 * N * V * D
+    case = types.SimpleNamespace(flops_per_step=flops,
+                                 p=types.SimpleNamespace(name="linear_ce_gpt2_8192x768x50257"))
+    # per step: 4 logits launches of 0.15 ms, 4 dX of 0.12 ms, 2 dW of 0.21 ms, 4 finalizes of 0.01 ms
+    kern = {"logits_gemm": (steps * 4 * 0.15, steps * 4), "dx_gemm": (steps * 4 * 0.12, steps * 4),
+            "dw_gemm": (steps * 2 * 0.21, steps * 2), "chunk_ce": (steps * 4 * 0.01, steps * 4)}
+    pk = dict(bench.FALLBACK_PEAKS)
+    step_ms = 1.6
+    r = bench.linear_roofline(case, step_ms * steps, kern, steps, pk, "fallback")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(flops / (step_ms * 1e-3) / 1e12)
+    assert r["peak"] == pk["bf16_tflops"] and "burst" in r["peak_source"]
+    assert r["frac"] == pytest.approx(r["achieved"] / pk["bf16_tflops"])
+    lg = r["kernels"]["logits_gemm"]
+    assert lg["launches_per_step"] == 4 and lg["ms_per_step"] == pytest.approx(0.6)
+    assert lg["tflops"] == pytest.approx(flops / 3 / 4 / (0.15e-3) / 1e12)
+    assert r["kernels"]["dw_gemm"]["tflops"] == pytest.approx(flops / 3 / 2 / (0.21e-3) / 1e12)
+    assert "tflops" not in r["kernels"]["chunk_ce"]
+    per = {k: bench.profiled_traffic(k, r["source_sha"], case.p.name) for k in bench.GEMM_KINDS}
+    if all(v is not None for v in per.values()):
+        assert r["traffic"] == pytest.approx(4 * per["logits_gemm"] + 4 * per["dx_gemm"] + 2 * per["dw_gemm"])
+    else:
+        assert r["traffic"] is None
+    # a timed region of two seconds or more is compared with the sustained peak
+    long = bench.linear_roofline(case, 2500.0, kern, steps, pk, "fallback")
+    assert long["peak"] == pk["bf16_tflops_sustained"] and "sustained" in long["peak_source"]
+
+
+def test_ce_roofline_is_algorithmic_bytes_over_the_kernel_time(monkeypatch):
+    """achieved = the step's algorithmic bytes (valid rows read once, every
+    gradient row written once, targets) over the CE kernel's mean launch time;
+    frac against the copy bandwidth; traffic looked up for the kernel's digest."""
+    import types
+    import bench
+    monkeypatch.setattr(bench, "ce_kernel_of",
+                        lambda case, dev: ("ce_ring2_kernel", ["lm_head_cross_gh_b200/csrc/ce_ring.cu",
+                                                                "lm_head_cross_gh_b200/csrc/ce_device.cuh",
+                                                                "lm_head_cross_gh_b200/csrc/common.cuh"]))
+    case = types.SimpleNamespace(bytes_per_step=1_630_503_130, op="fwd_bwd",
+                                 p=types.SimpleNamespace(name="ce_gpt2_bf16_8192x50257"))
+    pk = dict(bench.FALLBACK_PEAKS)
+    r = bench.ce_roofline(case, {"ce_row": (20 * 0.3, 20)}, 20, pk, "fallback", 0)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["kernel"] == "ce_ring2_kernel"
+    assert r["kernel_ms"] == pytest.approx(0.3)
+    assert r["achieved"] == pytest.approx(1_630_503_130 / 0.3e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / pk["hbm_gbs"]) and r["peak_source"] == "fallback (copy)"
+    assert r["traffic"] == bench.profiled_traffic("ce_ring2_kernel", r["source_sha"], case.p.name)
+
+
+def test_peaks_prefer_the_measured_file(monkeypatch, tmp_path):
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    pk, kind = bench.peaks()
+    assert kind == "fallback" and pk == bench.FALLBACK_PEAKS
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6543.4, "bf16_tflops": 1637.0}))
+    pk, kind = bench.peaks()
+    assert kind == "measured" and pk["hbm_gbs"] == 6543.4
