@@ -142,3 +142,22 @@ def test_peaks_prefer_the_measured_file(monkeypatch, tmp_path):
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6543.4, "bf16_tflops": 1637.0}))
     pk, kind = bench.peaks()
     assert kind == "measured" and pk["hbm_gbs"] == 6543.4
+
+
+def test_source_digest_ignores_comments_and_layout_only(tmp_path, monkeypatch):
+    """The digest that keys profiled DRAM traffic to the kernel source: a
+    comment or whitespace edit keeps it (a capture stays valid), any code edit
+    changes it (the capture no longer describes the kernel), and comment
+    markers inside string literals are code."""
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    src = ('// header comment\n__global__ void k(float* p) {\n  /* block\n comment */ p[0] = 1.0f;  // tail\n'
+           '  printf("// not a comment /* either */");\n}\n')
+    (tmp_path / "a.cu").write_text(src)
+    d0 = bench.source_digest(["a.cu"])
+    (tmp_path / "a.cu").write_text(src.replace("// header comment", "// reworded header").replace("  p[0]", "    p[0]"))
+    assert bench.source_digest(["a.cu"]) == d0
+    (tmp_path / "a.cu").write_text(src.replace("1.0f", "2.0f"))
+    assert bench.source_digest(["a.cu"]) != d0
+    (tmp_path / "a.cu").write_text(src.replace("/* either */", "/* neither */"))
+    assert bench.source_digest(["a.cu"]) != d0
